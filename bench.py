@@ -1,0 +1,403 @@
+#!/usr/bin/env python
+"""Benchmark of the routed-expert HFQ4 MoE layer on B200.
+
+Default workload: the decode stack of 40 MoE layers (hidden 2048, expert
+intermediate 512, 256 experts per layer, top-8, 1 token, bf16 residual
+stream), all experts resident in HBM.  A step is one token through all 40
+layers: route, gate/up GEMV with SiLU*up, down GEMV with the weighted
+combine, residual add.  Every step routes a different token (64 distinct
+tokens' logits cycled), so a step streams 535 MB of expert weights, more
+than the 126 MB L2: no flush is needed between steps.
+
+Prints one JSON line (rank 0).  --impl reference times the oracle (CPU,
+fp64) on bounded samples of the same workload instead.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "MoE-layer decode tokens/s and achieved GB/s as % of HBM/PCIe roofline"
+FALLBACK_HBM_GBS = 6650.0
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10000)
+    ap.add_argument("--warmup", type=int, default=50)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", choices=["decode"], default="decode")
+    ap.add_argument("--e2e-steps", type=int, default=2000)
+    ap.add_argument("--distinct-tokens", type=int, default=64)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--path", type=int, default=0, help="0 auto, 1 GEMV")
+    return ap.parse_args()
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return float(d["hbm_gbs"]), "measured"
+    return FALLBACK_HBM_GBS, "fallback"
+
+
+# ------------------------------------------------------------------ clocks
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    NAMES = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(prefix="clocks", suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        self.proc.wait()
+        sm, smax, reasons = [], [], set()
+        for line in open(self.path):
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax.append(float(f[2]))
+            except ValueError:
+                continue
+            for name, v in zip(self.NAMES, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(name)
+        os.unlink(self.path)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ------------------------------------------------------------- our arm
+
+def build_decode(torch, w, G):
+    import numpy as np
+
+    import expert_offload_b200 as eo
+    from expert_offload_b200.model import ExpertStore
+    import synth
+    from synth import workloads as W
+
+    def fill(l, g, u, d):
+        s = torch.cuda.current_stream().cuda_stream
+        E = g.shape[0]
+        synth.weights_dev(g.data_ptr(), w.seed, l, 0, E, synth.MAT_GATE, w.inter, w.hidden,
+                          W.WEIGHT_SIGMA, s)
+        synth.weights_dev(u.data_ptr(), w.seed, l, 0, E, synth.MAT_UP, w.inter, w.hidden,
+                          W.WEIGHT_SIGMA, s)
+        synth.weights_dev(d.data_ptr(), w.seed, l, 0, E, synth.MAT_DOWN, w.hidden, w.inter,
+                          W.WEIGHT_SIGMA, s)
+
+    store = ExpertStore(torch, w.layers, w.experts, w.hidden, w.inter, fill)
+    T = 1
+    logits = np.stack([W.logits_stack(w, g * T, T) for g in range(G)])          # [G, L, T, E]
+    xs = np.stack([W.activations(w, g * T, T)[0] for g in range(G)])            # [G, T, H] bf16
+    return eo, store, logits, xs
+
+
+def run_ours(args, rank, world, local_rank):
+    import numpy as np
+    import torch
+
+    torch.cuda.set_device(local_rank)
+    dist = None
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    from synth import workloads as W
+
+    w = W.WORKLOADS[2]
+    G = args.distinct_tokens
+    eo, store, logits, xs = build_decode(torch, w, G)
+    L, H, I, E, k, T = w.layers, w.hidden, w.inter, w.experts, w.top_k, 1
+    eb = eo.hfq4_expert_bytes(H, I)
+    d_logits = torch.from_numpy(logits).cuda()
+    d_x = torch.from_numpy(xs.view(np.int16)).cuda()
+    x_out = torch.empty((G, T, H), dtype=torch.int16, device="cuda")
+    ws = torch.zeros(eo.hfq4_stack_workspace_bytes(T, k, H, I, E), dtype=torch.uint8,
+                     device="cuda")
+    arr = eo.layer_array(store.layers)
+    stream = torch.cuda.Stream()
+
+    def step(g, s=None):
+        eo.hfq4_moe_decode_stack(store.layers, d_logits[g], k, d_x[g], T, x_out[g], ws,
+                                 path=args.path, stream=s, _layer_array=arr)
+
+    # graphs: one per distinct token (the persistent path is one launch per step
+    # either way; graphs remove host launch cost from the device timeline)
+    with torch.cuda.stream(stream):
+        for g in range(G):
+            step(g, stream)
+    torch.cuda.synchronize()
+    graphs = []
+    for g in range(G):
+        gr = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(gr, stream=stream):
+            step(g, stream)
+        graphs.append(gr)
+    torch.cuda.synchronize()
+    launches_per_step = eo_launches_per_step(eo, L)
+
+    with torch.cuda.stream(stream):
+        for i in range(args.warmup):
+            graphs[i % G].replay()
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    sampler = ClockSampler(local_rank)
+    sampler.start()
+    K = args.steps
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(K + 1)]
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    with torch.cuda.stream(stream):
+        ev[0].record(stream)
+        for i in range(K):
+            graphs[i % G].replay()
+            ev[i + 1].record(stream)
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    clocks = sampler.stop()
+    total_ms = ev[0].elapsed_time(ev[K])
+    per_launch = [ev[i].elapsed_time(ev[i + 1]) for i in range(K)]
+    eo.hfq_workspace_status(ws, stream)
+
+    # end to end through the C ABI: pinned host inputs copied in, result copied out
+    K2 = min(args.e2e_steps, K)
+    h_logits = torch.from_numpy(logits).pin_memory()
+    h_x = torch.from_numpy(xs.view(np.int16)).pin_memory()
+    h_out = torch.empty((G, T, H), dtype=torch.int16).pin_memory()
+    in_l = torch.empty_like(d_logits[0])
+    in_x = torch.empty_like(d_x[0])
+    out_x = torch.empty_like(x_out[0])
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        for i in range(min(20, K2)):
+            g = i % G
+            in_l.copy_(h_logits[g], non_blocking=True)
+            in_x.copy_(h_x[g], non_blocking=True)
+            eo.hfq4_moe_decode_stack(store.layers, in_l, k, in_x, T, out_x, ws, path=args.path,
+                                     stream=stream, _layer_array=arr)
+            h_out[g].copy_(out_x, non_blocking=True)
+        torch.cuda.synchronize()
+        e0.record(stream)
+        for i in range(K2):
+            g = i % G
+            in_l.copy_(h_logits[g], non_blocking=True)
+            in_x.copy_(h_x[g], non_blocking=True)
+            eo.hfq4_moe_decode_stack(store.layers, in_l, k, in_x, T, out_x, ws, path=args.path,
+                                     stream=stream, _layer_array=arr)
+            h_out[g].copy_(out_x, non_blocking=True)
+        e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1)
+
+    if dist:
+        t = torch.tensor([total_ms, e2e_ms], dtype=torch.float64, device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms, e2e_ms = float(t[0]), float(t[1])
+
+    bytes_per_step = L * k * eb * T      # T = 1: k unique experts per layer
+    value = world * K * T / (total_ms / 1e3)
+    mean_launch_ms = sum(per_launch) / K
+    achieved = bytes_per_step / (mean_launch_ms / 1e3) / 1e9
+    peak, peak_kind = peaks()
+    out = {
+        "metric": METRIC, "value": round(value, 2), "unit": "tokens/s", "n_gpus": world,
+        "steps": K, "warmup": args.warmup, "ms_per_step": round(total_ms / K, 5),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f32", "data": "synthetic",
+        "config": {"workload": w.name, "layers": L, "hidden": H, "inter": I, "experts": E,
+                   "top_k": k, "tokens_per_step": T, "weights": "hfq4 (136-byte blocks)",
+                   "activations": "bf16", "accumulate": "f32",
+                   "distinct_tokens_cycled": G, "bytes_per_step": bytes_per_step,
+                   "l2": "per-step working set 535 MB > 126 MB L2, no flush",
+                   "parallelism": f"replicas x{world}"},
+        "achieved_gbs": round(bytes_per_step * world * K / (total_ms / 1e3) / 1e9, 1),
+        "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak,
+                     "unit": "GB/s", "frac": round(achieved / peak, 4), "traffic": None,
+                     "peak_source": peak_kind,
+                     "kernel": "decode stack step (one launch sequence per token)",
+                     "bytes_per_launch": bytes_per_step,
+                     "mean_launch_ms": round(mean_launch_ms, 5)},
+        "e2e": {"value": round(world * K2 * T / (e2e_ms / 1e3), 2), "unit": "tokens/s",
+                "h2d_bytes_per_step": int(in_l.numel() * 4 + in_x.numel() * 2),
+                "d2h_bytes_per_step": int(out_x.numel() * 2)},
+        "gpu_launches": launches_per_step * K,
+        "clocks": clocks,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        out["cpu_baseline"] = cpu_baseline(w)
+    if dist:
+        dist.barrier()
+        graphs.clear()
+        dist.destroy_process_group()
+    store.close()
+    return out
+
+
+def eo_launches_per_step(eo, L):
+    # route + gate/up + down per layer for the per-layer path
+    return 3 * L
+
+
+# ------------------------------------------------------- oracle (CPU) arms
+
+def _threads_one():
+    try:
+        from threadpoolctl import threadpool_limits
+        return threadpool_limits(1)
+    except ImportError:
+        return None
+
+
+def cpu_baseline(w, layers_sampled: int = 3):
+    """The oracle as it stands, single-threaded, on one token through the
+    first `layers_sampled` layers of the stack (dequantise the selected
+    experts' HFQ4 bytes and run them in fp64); packing is load time and is
+    not timed.  tokens/s = 1 / (time per layer x L)."""
+    import numpy as np
+
+    from oracle import hfq4, moe, route
+    from synth import workloads as W
+
+    lim = _threads_one()
+    x = W.activations_value(w, 0, 1)
+    packed, routes = [], []
+    for l in range(layers_sampled):
+        lg = W.logits(w, l, 0, 1)
+        idx, wts = route.route(lg, w.top_k)
+        ex = {int(e): hfq4.pack_expert(*W.expert_matrices(w, l, int(e))) for e in idx[0]}
+        packed.append(ex)
+        routes.append((lg, idx, wts))
+    t0 = time.perf_counter()
+    for l in range(layers_sampled):
+        idx, wts = route.route(routes[l][0], w.top_k)
+        cache = moe.ExpertCache(packed[l], w.hidden, w.inter)
+        y = moe.moe_layer(cache, w.hidden, w.inter, x, idx, wts)
+        x = moe.round_bf16(x + y)
+    dt = time.perf_counter() - t0
+    if lim is not None:
+        lim.unregister() if hasattr(lim, "unregister") else None
+    return {"value": round(layers_sampled / (dt * w.layers), 6), "unit": "tokens/s", "cores": 1,
+            "kind": "oracle",
+            "sample": f"1 token through layers 0..{layers_sampled - 1} of the {w.layers}-layer "
+                      f"stack ({layers_sampled * w.top_k} expert FFNs, HFQ4 dequantise + fp64 "
+                      f"GEMVs), {dt:.1f} s, scaled by {w.layers}/{layers_sampled}"}
+
+
+def run_reference(args):
+    """The oracle as the reference arm: each step runs the oracle's HFQ4
+    dequantise + fp64 GEMV over a bounded byte sample of one token's work
+    (rows of the selected experts of a layer), sized so that the whole run
+    stays within a few minutes; tokens/s = bytes/s / bytes per token."""
+    import numpy as np
+
+    from oracle import hfq4, moe, route
+    from synth import workloads as W
+
+    lim = _threads_one()
+    w = W.WORKLOADS[2]
+    H, I, k, L = w.hidden, w.inter, w.top_k, w.layers
+    eb = hfq4.expert_bytes(H, I)
+    bytes_per_token = L * k * eb
+    idx, wts = route.route(W.logits(w, 0, 0, 1), k)
+    experts = [hfq4.pack_expert(*W.expert_matrices(w, 0, int(e))) for e in idx[0][:2]]
+    x = W.activations_value(w, 0, 1)[0]
+    row_bytes = hfq4.matrix_bytes(1, H)
+    budget = min(0.5, 150.0 / max(1, args.steps + args.warmup))
+    # calibrate rows per step on 64 gate rows
+    t0 = time.perf_counter()
+    hfq4.dequantize_exact(experts[0][:64 * row_bytes], 64, H) @ x
+    per_row = (time.perf_counter() - t0) / 64
+    rows = int(max(1, min(I, budget / max(per_row, 1e-9))))
+
+    def one_step(i):
+        ex = experts[i % len(experts)]
+        r0 = (i * rows) % (I - rows + 1) if rows < I else 0
+        g = hfq4.dequantize_exact(ex[r0 * row_bytes:(r0 + rows) * row_bytes], rows, H) @ x
+        mg = hfq4.matrix_bytes(I, H)
+        u = hfq4.dequantize_exact(ex[mg + r0 * row_bytes:mg + (r0 + rows) * row_bytes], rows, H) @ x
+        return moe.silu(g) * u
+
+    for i in range(args.warmup):
+        one_step(i)
+    t0 = time.perf_counter()
+    for i in range(args.steps):
+        one_step(i)
+    dt = time.perf_counter() - t0
+    bytes_done = args.steps * 2 * rows * row_bytes
+    value = bytes_done / dt / bytes_per_token
+    return {"impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": "tokens/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(dt / args.steps * 1e3, 4), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": w.name, "layers": L, "hidden": H, "inter": I,
+                       "experts": w.experts, "top_k": k, "tokens_per_step": 1},
+            "cpu_baseline": {"value": round(value, 6), "unit": "tokens/s", "cores": 1,
+                             "kind": "oracle",
+                             "sample": f"each step: {rows} gate + {rows} up rows of one selected "
+                                       f"expert (HFQ4 dequantise + fp64 GEMV + SiLU*up); "
+                                       f"tokens/s = HFQ4 bytes/s / {bytes_per_token} bytes per "
+                                       f"token"},
+            "e2e": {"value": round(value, 6), "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+
+
+def main():
+    args = parse()
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", str(args.gpus)))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if "WORLD_SIZE" not in os.environ:
+        world = 1
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        print(json.dumps(run_reference(args)), flush=True)
+        return
+    out = run_ours(args, rank, world, local_rank)
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+
+
+if __name__ == "__main__":
+    main()

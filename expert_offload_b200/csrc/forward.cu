@@ -1,0 +1,313 @@
+// forward.cu - the routed-expert HFQ4 GEMV path (decode and speculative
+// verify): gate/up GEMV with fused SiLU(gate)*up, then the down GEMV with the
+// weighted combine fused into it.  Entry points hfq4_moe_forward and
+// hfq4_moe_decode_stack.
+//
+// hipfire thread, "HFQ quantisation format and GEMV": decode is a GEMV over
+// 136-byte blocks and bandwidth-bound.  Each warp owns output rows; lanes
+// split a row's blocks into 8-byte chunks of 16 nibbles and reduce with warp
+// shuffles; per block the dot product is factored as
+//     sum_i (zero + scale*q_i) x_i = scale * sum_i q_i x_i + zero * sum_i x_i.
+#include <cfloat>
+
+#include "device.cuh"
+
+namespace hfq {
+namespace {
+
+constexpr int kThreads = 256;            // 8 warps
+constexpr int kWarps = kThreads / 32;
+constexpr int kRowsPerWarp = 4;
+constexpr int kRowsPerCta = kWarps * kRowsPerWarp;
+constexpr size_t kMaxDownSmem = 192 * 1024;   // k * ceil(I/256) <= 192 staged h vectors
+
+// Dot product of one HFQ4 row (nb blocks) with a zero-padded f32 vector in
+// shared memory.  Returns the full sum in every lane.
+__device__ __forceinline__ float row_dot(const uint8_t *__restrict__ row, int nb,
+                                         const float *__restrict__ xs)
+{
+    float acc = 0.0f;
+    for (int c = threadIdx.x & 31; c < nb * 16; c += 32) {
+        const int b = c >> 4, j = c & 15;
+        const uint8_t *blk = row + (size_t)b * kBlockBytes;
+        const float2 sz = *reinterpret_cast<const float2 *>(blk);       // scale, zero
+        const uint2 nib = *reinterpret_cast<const uint2 *>(blk + 8 + j * 8);
+        const float *xp = xs + b * kBlock + j * 16;
+        float sq = 0.0f, sx = 0.0f;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            float x0 = xp[i], x1 = xp[8 + i];
+            sq = fmaf((float)((nib.x >> (4 * i)) & 15u), x0, sq);
+            sq = fmaf((float)((nib.y >> (4 * i)) & 15u), x1, sq);
+            sx += x0 + x1;
+        }
+        acc = fmaf(sz.x, sq, fmaf(sz.y, sx, acc));
+    }
+    return warp_sum(acc);
+}
+
+// Gate/up: CTA (pair p = t*k + j, row chunk).  h[p][r] = silu(g_r) * u_r.
+__global__ void __launch_bounds__(kThreads)
+gateup_kernel(const void *const *__restrict__ eptr, const void *__restrict__ x, int x_dtype,
+              const int32_t *__restrict__ idx, int k, int H, int I, float *__restrict__ h)
+{
+    extern __shared__ float xs[];               // [nbH * 256]
+    const int p = blockIdx.x, t = p / k;
+    const int nbH = (H + kBlock - 1) / kBlock;
+    for (int i = threadIdx.x; i < nbH * kBlock; i += kThreads)
+        xs[i] = i < H ? load_act(x, x_dtype, (size_t)t * H + i) : 0.0f;
+    __syncthreads();
+    const uint8_t *base = static_cast<const uint8_t *>(eptr[idx[p]]);
+    const size_t row_bytes = (size_t)nbH * kBlockBytes;
+    const uint8_t *gate = base, *up = base + (size_t)I * row_bytes;
+    const int warp = threadIdx.x >> 5;
+    const int nbI = (I + kBlock - 1) / kBlock;
+    for (int rr = 0; rr < kRowsPerWarp; ++rr) {
+        const int r = blockIdx.y * kRowsPerCta + warp * kRowsPerWarp + rr;
+        if (r >= I) break;
+        float g = row_dot(gate + r * row_bytes, nbH, xs);
+        float u = row_dot(up + r * row_bytes, nbH, xs);
+        if ((threadIdx.x & 31) == 0) h[(size_t)p * nbI * kBlock + r] = silu(g) * u;
+    }
+}
+
+// Down + combine: CTA (token t, row chunk).  y[t][r] = sum_j w_j * Wd_ej[r] . h[t,j].
+// With x_res != null also writes x_next[t][r] = bf16(x_res[t][r] + y[t][r]).
+__global__ void __launch_bounds__(kThreads)
+down_kernel(const void *const *__restrict__ eptr, const float *__restrict__ h,
+            const int32_t *__restrict__ idx, const float *__restrict__ wts, int k, int H, int I,
+            float *__restrict__ y, uint16_t *__restrict__ y_bf16,
+            const uint16_t *__restrict__ x_res, uint16_t *__restrict__ x_next)
+{
+    extern __shared__ float hs[];               // [k][nbI * 256]
+    const int t = blockIdx.x;
+    const int nbI = (I + kBlock - 1) / kBlock, hl = nbI * kBlock;
+    for (int i = threadIdx.x; i < k * hl; i += kThreads) {
+        int j = i / hl, c = i - j * hl;
+        hs[i] = c < I ? h[((size_t)t * k + j) * hl + c] : 0.0f;
+    }
+    __syncthreads();
+    const int nbH = (H + kBlock - 1) / kBlock;
+    const size_t gate_bytes = (size_t)I * nbH * kBlockBytes;
+    const size_t row_bytes = (size_t)nbI * kBlockBytes;
+    const int warp = threadIdx.x >> 5;
+    for (int rr = 0; rr < kRowsPerWarp; ++rr) {
+        const int r = blockIdx.y * kRowsPerCta + warp * kRowsPerWarp + rr;
+        if (r >= H) break;
+        float acc = 0.0f;
+        for (int j = 0; j < k; ++j) {
+            const uint8_t *down =
+                static_cast<const uint8_t *>(eptr[idx[(size_t)t * k + j]]) + 2 * gate_bytes;
+            float o = row_dot(down + (size_t)r * row_bytes, nbI, hs + j * hl);
+            acc = fmaf(wts[(size_t)t * k + j], o, acc);
+        }
+        if ((threadIdx.x & 31) == 0) {
+            size_t o = (size_t)t * H + r;
+            if (y) y[o] = acc;
+            if (y_bf16) y_bf16[o] = float_to_bf16_bits(acc);
+            if (x_next) x_next[o] = float_to_bf16_bits(bf16_bits_to_float(x_res[o]) + acc);
+        }
+    }
+}
+
+// Per-layer route for the decode stack (T <= 8 tokens, one warp each).
+__global__ void stack_route_kernel(const float *__restrict__ logits, int T, int E, int k,
+                                   int32_t *__restrict__ idx, float *__restrict__ wts,
+                                   int32_t *__restrict__ idx_out, float *__restrict__ wts_out)
+{
+    const int t = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (t >= T) return;
+    const float *l = logits + (size_t)t * E;
+    // each lane keeps a bitmask of its selected experts (E <= 512 -> 16 per lane)
+    uint32_t mine = 0;
+    int sel[HFQ_MAX_TOPK];
+    float sv[HFQ_MAX_TOPK];
+    for (int j = 0; j < k; ++j) {
+        float bv = -INFINITY;
+        int bi = 0x7fffffff;
+        for (int s = 0, e = lane; e < E; ++s, e += 32) {
+            if (mine >> s & 1u) continue;
+            float v = l[e];
+            if (v > bv || (v == bv && e < bi)) { bv = v; bi = e; }
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+            int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+            if (ov > bv || (ov == bv && oi < bi)) { bv = ov; bi = oi; }
+        }
+        sel[j] = bi;
+        sv[j] = bv;
+        if ((bi & 31) == lane) mine |= 1u << (bi >> 5);
+    }
+    if (lane == 0) {
+        float s = 0.0f, ex[HFQ_MAX_TOPK];
+        for (int j = 0; j < k; ++j) { ex[j] = __expf(sv[j] - sv[0]); s += ex[j]; }
+        for (int j = 0; j < k; ++j) {
+            float w = ex[j] / s;
+            idx[t * k + j] = sel[j];
+            wts[t * k + j] = w;
+            if (idx_out) { idx_out[t * k + j] = sel[j]; wts_out[t * k + j] = w; }
+        }
+    }
+}
+
+size_t h_bytes(int T, int k, int I)
+{
+    size_t nbI = (I + kBlock - 1) / kBlock;
+    return ((size_t)T * k * nbI * kBlock * sizeof(float) + 255) / 256 * 256;
+}
+
+size_t act_bytes(int T, int H) { return ((size_t)T * H * 2 + 255) / 256 * 256; }
+
+hfq_status check_ws(void *ws, size_t ws_bytes, size_t need)
+{
+    if (!ws || ws_bytes < need)
+        return fail(HFQ_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", need, ws_bytes);
+    if ((uintptr_t)ws & 255) return fail(HFQ_ERR_ALIGN, "workspace must be 256-byte aligned");
+    return HFQ_OK;
+}
+
+hfq_status launch_layer(const hfq4_layer &L, const void *x, int x_dtype, int T, const int32_t *idx,
+                        const float *wts, int k, float *y, void *y_bf16, float *h,
+                        const uint16_t *x_res, uint16_t *x_next, cudaStream_t s)
+{
+    const int H = L.hidden, I = L.inter;
+    const int nbH = (H + kBlock - 1) / kBlock, nbI = (I + kBlock - 1) / kBlock;
+    const size_t smem_down = (size_t)k * nbI * kBlock * sizeof(float);
+    if (smem_down > kMaxDownSmem)
+        return fail(HFQ_ERR_UNSUPPORTED, "k * ceil(inter/256) = %d exceeds %d", k * nbI,
+                    (int)(kMaxDownSmem / 1024));
+    static bool attr_set = false;
+    if (!attr_set) {
+        cudaFuncSetAttribute(down_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)kMaxDownSmem);
+        attr_set = true;
+    }
+    dim3 g1(T * k, (I + kRowsPerCta - 1) / kRowsPerCta);
+    gateup_kernel<<<g1, kThreads, nbH * kBlock * sizeof(float), s>>>(
+        L.expert_ptr, x, x_dtype, idx, k, H, I, h);
+    dim3 g2(T, (H + kRowsPerCta - 1) / kRowsPerCta);
+    down_kernel<<<g2, kThreads, smem_down, s>>>(
+        L.expert_ptr, h, idx, wts, k, H, I, y, static_cast<uint16_t *>(y_bf16), x_res, x_next);
+    cudaError_t err = cudaGetLastError();
+    if (err != cudaSuccess) return fail(HFQ_ERR_CUDA, "forward launch: %s", cudaGetErrorString(err));
+    return HFQ_OK;
+}
+
+hfq_status check_layer(const hfq4_layer *layer, int k)
+{
+    if (!layer || !layer->expert_ptr) return fail(HFQ_ERR_ARG, "layer or expert_ptr is null");
+    return check_shape(layer->hidden, layer->inter, layer->n_experts, k);
+}
+
+}  // namespace
+}  // namespace hfq
+
+using namespace hfq;
+
+extern "C" {
+
+size_t hfq4_moe_workspace_bytes(int T, int k, int hidden, int inter, int n_experts)
+{
+    if (T < 1 || k < 1 || hidden < 1 || inter < 1 || n_experts < 1) return 0;
+    return kWsHeader + h_bytes(T, k, inter);
+}
+
+hfq_status hfq4_moe_forward(const hfq4_layer *layer, const void *x, hfq_dtype x_dtype, int T,
+                            const int32_t *idx, const float *wts, int k, const int32_t *cnt,
+                            const int32_t *off, const int32_t *perm, float *y, void *y_bf16,
+                            int path, void *workspace, size_t ws_bytes, void *stream)
+{
+    (void)cnt; (void)off; (void)perm;
+    hfq_status st = check_layer(layer, k);
+    if (st) return st;
+    if (!x || !idx || !wts || !y) return fail(HFQ_ERR_ARG, "hfq4_moe_forward: null pointer");
+    if (T < 1 || T > 65536) return fail(HFQ_ERR_UNSUPPORTED, "T=%d not in [1, 65536]", T);
+    if (x_dtype != HFQ_F32 && x_dtype != HFQ_BF16) return fail(HFQ_ERR_ARG, "bad x_dtype");
+    if (path != HFQ_PATH_AUTO && path != HFQ_PATH_GEMV)
+        return fail(HFQ_ERR_UNSUPPORTED, "path %d is not available in this build", path);
+    if (!aligned16(x) || !aligned16(y) || (y_bf16 && !aligned16(y_bf16)))
+        return fail(HFQ_ERR_ALIGN, "x, y and y_bf16 must be 16-byte aligned");
+    size_t need = hfq4_moe_workspace_bytes(T, k, layer->hidden, layer->inter, layer->n_experts);
+    if ((st = check_ws(workspace, ws_bytes, need))) return st;
+    float *h = reinterpret_cast<float *>(static_cast<char *>(workspace) + kWsHeader);
+    st = launch_layer(*layer, x, x_dtype, T, idx, wts, k, y, y_bf16, h, nullptr, nullptr,
+                      (cudaStream_t)stream);
+    return st ? st : ok();
+}
+
+size_t hfq4_stack_workspace_bytes(int T, int k, int hidden, int inter, int n_experts)
+{
+    if (T < 1 || T > 8 || k < 1 || hidden < 1 || inter < 1 || n_experts < 1) return 0;
+    return kWsHeader + h_bytes(T, k, inter) + 2 * act_bytes(T, hidden) +
+           ((size_t)T * k * 8 + 255) / 256 * 256;
+}
+
+hfq_status hfq4_moe_decode_stack(const hfq4_layer *layers, int n_layers, const float *logits,
+                                 int k, const void *x0, int T, void *x_out, float *y_all,
+                                 int32_t *idx_all, float *wts_all, int path, void *workspace,
+                                 size_t ws_bytes, void *stream)
+{
+    if (!layers || n_layers < 1 || n_layers > HFQ_MAX_STACK_LAYERS)
+        return fail(HFQ_ERR_ARG, "n_layers=%d not in [1, %d]", n_layers, HFQ_MAX_STACK_LAYERS);
+    hfq_status st;
+    for (int l = 0; l < n_layers; ++l) {
+        if ((st = check_layer(&layers[l], k))) return st;
+        if (layers[l].hidden != layers[0].hidden || layers[l].inter != layers[0].inter ||
+            layers[l].n_experts != layers[0].n_experts)
+            return fail(HFQ_ERR_ARG, "layer %d has a different shape", l);
+    }
+    if (!logits || !x0 || !x_out) return fail(HFQ_ERR_ARG, "null pointer");
+    if (T < 1 || T > 8) return fail(HFQ_ERR_UNSUPPORTED, "decode stack takes T in [1, 8], got %d", T);
+    if ((idx_all == nullptr) != (wts_all == nullptr))
+        return fail(HFQ_ERR_ARG, "idx_all and wts_all go together");
+    if (path != HFQ_PATH_AUTO && path != HFQ_PATH_GEMV)
+        return fail(HFQ_ERR_UNSUPPORTED, "decode stack runs the GEMV path only");
+    if (!aligned16(x0) || !aligned16(x_out) || (y_all && !aligned16(y_all)))
+        return fail(HFQ_ERR_ALIGN, "x0, x_out and y_all must be 16-byte aligned");
+    const int H = layers[0].hidden, I = layers[0].inter, E = layers[0].n_experts;
+    size_t need = hfq4_stack_workspace_bytes(T, k, H, I, E);
+    if ((st = check_ws(workspace, ws_bytes, need))) return st;
+    char *ws = static_cast<char *>(workspace) + kWsHeader;
+    float *h = reinterpret_cast<float *>(ws);
+    ws += h_bytes(T, k, I);
+    uint16_t *xa = reinterpret_cast<uint16_t *>(ws);
+    ws += act_bytes(T, H);
+    uint16_t *xb = reinterpret_cast<uint16_t *>(ws);
+    ws += act_bytes(T, H);
+    int32_t *idx = reinterpret_cast<int32_t *>(ws);
+    float *wts = reinterpret_cast<float *>(ws + (size_t)T * k * 4);
+    cudaStream_t s = (cudaStream_t)stream;
+    const uint16_t *cur = static_cast<const uint16_t *>(x0);
+    for (int l = 0; l < n_layers; ++l) {
+        uint16_t *next = (l == n_layers - 1) ? static_cast<uint16_t *>(x_out) : (l & 1 ? xb : xa);
+        stack_route_kernel<<<1, 32 * T, 0, s>>>(logits + (size_t)l * T * E, T, E, k, idx, wts,
+                                                idx_all ? idx_all + (size_t)l * T * k : nullptr,
+                                                wts_all ? wts_all + (size_t)l * T * k : nullptr);
+        float *y = y_all ? y_all + (size_t)l * T * H : nullptr;
+        st = launch_layer(layers[l], cur, HFQ_BF16, T, idx, wts, k, y, nullptr, h, cur, next, s);
+        if (st) return st;
+        cur = next;
+    }
+    return ok();
+}
+
+hfq_status hfq_workspace_status(void *workspace, size_t ws_bytes, void *stream)
+{
+    if (!workspace || ws_bytes < kWsHeader) return fail(HFQ_ERR_ARG, "no workspace");
+    unsigned int word = 0;
+    cudaStream_t s = (cudaStream_t)stream;
+    cudaError_t err = cudaMemcpyAsync(&word, workspace, sizeof word, cudaMemcpyDeviceToHost, s);
+    if (err == cudaSuccess) err = cudaStreamSynchronize(s);
+    if (err != cudaSuccess) return fail(HFQ_ERR_CUDA, "status read: %s", cudaGetErrorString(err));
+    if (word != 0) {
+        unsigned int zero = 0;
+        cudaMemcpyAsync(workspace, &zero, sizeof zero, cudaMemcpyHostToDevice, s);
+        cudaStreamSynchronize(s);
+        return fail((hfq_status)(int)word, "a device-side wait ran out (status %d)", (int)word);
+    }
+    return ok();
+}
+
+}  // extern "C"

@@ -1,0 +1,264 @@
+/*
+ * hfq4moe.h - C ABI of libhfq4moe.so: the routed-expert MoE layer of LLM
+ * decode over HFQ4 block-quantised expert weights, on NVIDIA B200 (sm_100a).
+ *
+ * Sources (page title and section):
+ *   [HFQ]   hipfire RDNA engine forum thread, section "HFQ quantisation format
+ *           and GEMV optimisation": 256-weight blocks of 136 bytes, an f32
+ *           scale, an f32 zero point and 128 bytes of packed 4-bit data;
+ *           decode is a bandwidth-bound GEMV over such blocks.
+ *   [TOPK]  hipfire MoE expert-offload explainer, opening section: each token
+ *           activates 8 of its layer's experts (top-8 routing).
+ *   [PLACE] same explainer, section "placement algorithm": layer split
+ *           VRAM_LAYERS=N, auto fit-capacity placement, expert hot set, loud
+ *           refusal naming the byte deficit.
+ *   [PCIE]  same explainer, section "PCIe pass-through": host-mapped pinned
+ *           expert weights are read by the GPU kernel directly over PCIe,
+ *           with no staging copy.
+ *   [TABLE] Strata user report, section "model and engine": a per-(layer,
+ *           expert) offset table locates every expert's gate/up/down bytes.
+ *   [ARENA] Strata user report, pitfall 7: the pinned expert arena is
+ *           registered with the CUDA runtime, 2 MiB pages when available.
+ *   [WMMA]  gfx1151 engine README, Windows section: a self-written matrix-
+ *           core GEMM for prefill (prior art for the tensor-core path).
+ *
+ * Conventions shared by every entry point:
+ *   - Weights: w = zero + scale * q with q in [0, 15].  Block layout: f32
+ *     scale, f32 zero (little-endian), 128 bytes of nibbles, byte j holding
+ *     element 2j in its low nibble and 2j+1 in its high nibble.  A matrix of
+ *     R rows x C columns is R x ceil(C/256) blocks, row after row; a row
+ *     shorter than a whole number of blocks is padded with q = 0.
+ *   - A packed expert is [gate I x H][up I x H][down H x I] matrices, back
+ *     to back (hfq4_expert_bytes(H, I) bytes).  At H = 2048, I = 512 that is
+ *     1,671,168 bytes, a multiple of 256.
+ *   - Ownership: the caller allocates and owns every buffer (device memory
+ *     normally comes from the caller's allocator).  The library allocates
+ *     only the pinned host arenas that hfq_host_arena_create makes, and
+ *     never allocates on the forward path: scratch is the caller's
+ *     workspace, sized by the *_workspace_bytes queries.
+ *   - Streams: `stream` is a cudaStream_t passed as void*; NULL means the
+ *     legacy default stream.  GPU work is asynchronous on it.
+ *   - Errors: every call returns an hfq_status; argument errors are found on
+ *     the host before anything is launched and leave outputs untouched.
+ *     hfq_last_error() returns a thread-local message for the last failure.
+ *     Device-side conditions (a bounded wait that ran out) are written to a
+ *     status word in the workspace and read by hfq_workspace_status().
+ *   - Limits: 1 <= k <= 16, k <= E <= 512, H and I multiples of 128
+ *     (H, I <= 8192), T <= 65536, pointers 16-byte aligned.
+ */
+#ifndef HFQ4MOE_H
+#define HFQ4MOE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    HFQ_OK = 0,
+    HFQ_ERR_ARG = -1,          /* a size, count or pointer argument is invalid */
+    HFQ_ERR_ALIGN = -2,        /* a pointer is not 16-byte aligned */
+    HFQ_ERR_UNSUPPORTED = -3,  /* a shape outside the limits above */
+    HFQ_ERR_NOFIT = -4,        /* placement does not fit the HBM budget */
+    HFQ_ERR_CUDA = -5,         /* a CUDA runtime call failed */
+    HFQ_ERR_TIMEOUT = -6,      /* a bounded device-side wait ran out */
+    HFQ_ERR_ALLOC = -7,        /* host arena allocation or registration failed */
+    HFQ_ERR_WORKSPACE = -8     /* workspace missing or smaller than required */
+} hfq_status;
+
+typedef enum { HFQ_F32 = 0, HFQ_BF16 = 1 } hfq_dtype;
+
+/* Which expert path hfq4_moe_forward runs. */
+typedef enum {
+    HFQ_PATH_AUTO = 0,  /* GEMV when tokens per expert are few, else tensor cores */
+    HFQ_PATH_GEMV = 1,  /* CUDA-core HFQ4 GEMV (decode, speculative verify) */
+    HFQ_PATH_TC = 2     /* dequantise to bf16 + tcgen05 grouped GEMM (prefill) */
+} hfq_path;
+
+#define HFQ4_BLOCK 256
+#define HFQ4_BLOCK_BYTES 136
+#define HFQ_MAX_EXPERTS 512
+#define HFQ_MAX_TOPK 16
+#define HFQ_MAX_STACK_LAYERS 64
+
+/* Message of the last failed call on this thread ("" if none). */
+const char *hfq_last_error(void);
+
+/* Library version, major * 10000 + minor * 100 + patch. */
+int hfq_version(void);
+
+/* Bytes of an HFQ4 matrix [HFQ]: rows * ceil(cols / 256) * 136.  0 on bad args. */
+size_t hfq4_matrix_bytes(int rows, int cols);
+
+/* Bytes of one packed expert: 2 * matrix(I, H) + matrix(H, I).  0 on bad args. */
+size_t hfq4_expert_bytes(int hidden, int inter);
+
+/*
+ * Quantise and pack experts on the host [HFQ].
+ *   gate, up: f32 [n_experts][inter][hidden], row-major, host memory.
+ *   down:     f32 [n_experts][hidden][inter].
+ *   out:      host buffer of at least n_experts * hfq4_expert_bytes(hidden,
+ *             inter) bytes; expert e starts at e * hfq4_expert_bytes.
+ * Per block (the real elements of a row only): scale = f32(f32(max - min) /
+ * 15), zero = min, q = clamp(rint(f32(f32(w - zero) / scale)), 0, 15),
+ * rounding half to even; scale == 0 stores q = 0.  Inputs must be finite.
+ * Single-threaded, deterministic, bit-identical to the device variant.
+ */
+hfq_status hfq4_pack_experts(const float *gate, const float *up, const float *down,
+                             int n_experts, int hidden, int inter, void *out, size_t out_bytes);
+
+/* Same as hfq4_pack_experts with device pointers, asynchronous on `stream`. */
+hfq_status hfq4_pack_experts_device(const float *gate, const float *up, const float *down,
+                                    int n_experts, int hidden, int inter, void *out,
+                                    size_t out_bytes, void *stream);
+
+/*
+ * Dequantise one HFQ4 matrix (device) [HFQ]: out[r][c] = fmaf(scale, q, zero),
+ * the correctly rounded f32 of zero + scale*q, for r < rows, c < cols.
+ *   blocks: device, hfq4_matrix_bytes(rows, cols) bytes, 8-byte aligned.
+ *   out:    device f32 [rows][cols].
+ */
+hfq_status hfq4_dequant(const void *blocks, int rows, int cols, float *out, void *stream);
+
+/*
+ * Top-k softmax routing with renormalised weights [TOPK] (device).
+ *   logits: f32 [T][E].
+ *   idx:    int32 [T][k] out: the k experts with the largest logits, slot 0
+ *           the largest; equal logits go to the lower expert index.
+ *   wts:    f32 [T][k] out: p_j / sum_selected p, p = softmax(logits); this
+ *           is the softmax over the selected logits.
+ *   cnt, off, perm: optional grouping by expert (all three or none):
+ *           cnt int32 [E] pairs per expert, off int32 [E+1] exclusive prefix
+ *           sum, perm int32 [T*k] the pair ids t*k+j of expert e at
+ *           perm[off[e] .. off[e+1]), ascending.
+ *   workspace: needed only with grouping, hfq_route_workspace_bytes(T, E, k)
+ *           bytes of device scratch (may be NULL when that is 0).
+ * NaN logits are not supported.
+ */
+size_t hfq_route_workspace_bytes(int T, int E, int k);
+hfq_status moe_route(const float *logits, int T, int E, int k, int32_t *idx, float *wts,
+                     int32_t *cnt, int32_t *off, int32_t *perm, void *workspace,
+                     size_t ws_bytes, void *stream);
+
+/*
+ * One MoE layer's experts [TABLE][PCIE].
+ *   expert_ptr: DEVICE array [n_experts] of base addresses of the packed
+ *               experts, each 16-byte aligned; an address may be HBM or a
+ *               host-mapped pinned buffer (see hfq_host_arena_create).
+ *   expert_loc: DEVICE array [n_experts] (or NULL = all HBM): 0 = HBM,
+ *               1 = host-mapped.  Host-mapped experts are read over PCIe by
+ *               the same kernel, with plain loads.
+ */
+typedef struct {
+    const void *const *expert_ptr;
+    const uint8_t *expert_loc;
+    int n_experts;
+    int hidden;
+    int inter;
+} hfq4_layer;
+
+/*
+ * Routed experts of one layer for T tokens (device):
+ *   y[t] = sum_j wts[t][j] * Wd_e (silu(Wg_e x_t) * (Wu_e x_t)),  e = idx[t][j],
+ * summed in slot order j with fp32 accumulation.
+ *   x:      [T][H] in x_dtype (f32 or bf16).
+ *   idx, wts: routing as written by moe_route ([T][k]).
+ *   cnt, off, perm: grouping by expert; required for HFQ_PATH_TC and AUTO
+ *           with T > 8, ignored otherwise (may be NULL).
+ *   y:      f32 [T][H] out.  y_bf16: optional bf16 [T][H] out (NULL = none).
+ *   workspace: hfq4_moe_workspace_bytes(T, k, H, I, E) bytes of device
+ *           scratch, 256-byte aligned, owned by the caller; calls that share
+ *           a workspace must be ordered on one stream.
+ */
+size_t hfq4_moe_workspace_bytes(int T, int k, int hidden, int inter, int n_experts);
+hfq_status hfq4_moe_forward(const hfq4_layer *layer, const void *x, hfq_dtype x_dtype, int T,
+                            const int32_t *idx, const float *wts, int k, const int32_t *cnt,
+                            const int32_t *off, const int32_t *perm, float *y, void *y_bf16,
+                            int path, void *workspace, size_t ws_bytes, void *stream);
+
+/*
+ * A decode stack of MoE layers joined by a bf16 residual stream (device):
+ * for l = 0 .. n_layers-1, route layer l on logits[l] (top-k softmax,
+ * renormalised), run its experts on x_l, then x_{l+1} = bf16(x_l + y_l).
+ * Layer l's logits are read only after layer l-1 has finished, as a router
+ * that depends on x_l would require.  One kernel per layer, or one
+ * persistent kernel for the whole stack (HFQ_PATH_AUTO/GEMV).
+ *   layers:  host array [n_layers] of layer descriptors (n_layers <= 64),
+ *            all with the same n_experts, hidden, inter.
+ *   logits:  f32 [n_layers][T][E] (device).
+ *   x0:      bf16 [T][H] (device), the residual stream entering layer 0.
+ *   x_out:   bf16 [T][H] out, the residual after the last layer (may alias
+ *            nothing else).
+ *   y_all:   optional f32 [n_layers][T][H] out: every layer's y (NULL = none).
+ *   idx_all, wts_all: optional int32/f32 [n_layers][T][k] out (NULL = none).
+ *   T <= 8.  workspace: hfq4_stack_workspace_bytes(T, k, H, I, E) bytes.
+ */
+size_t hfq4_stack_workspace_bytes(int T, int k, int hidden, int inter, int n_experts);
+hfq_status hfq4_moe_decode_stack(const hfq4_layer *layers, int n_layers, const float *logits,
+                                 int k, const void *x0, int T, void *x_out, float *y_all,
+                                 int32_t *idx_all, float *wts_all, int path, void *workspace,
+                                 size_t ws_bytes, void *stream);
+
+/*
+ * Device status word of a workspace (synchronises `stream`): HFQ_OK, or
+ * HFQ_ERR_TIMEOUT if a bounded device-side wait of a previous call ran out.
+ * The word is cleared by the read.
+ */
+hfq_status hfq_workspace_status(void *workspace, size_t ws_bytes, void *stream);
+
+/*
+ * Pinned, mapped host arena for offloaded experts [PCIE][ARENA].
+ *   bytes:   arena size.
+ *   flags:   HFQ_ARENA_HUGEPAGE asks for 2 MiB transparent huge pages
+ *            (madvise) before registration; it silently falls back to 4 KiB.
+ *   host:    out, host address of the arena.
+ *   dev:     out, the device address of the same memory (for expert_ptr).
+ * Returns HFQ_ERR_ALLOC with the byte count in the message when pinning fails.
+ * The library owns the arena until hfq_host_arena_destroy(host).
+ */
+#define HFQ_ARENA_HUGEPAGE 1
+hfq_status hfq_host_arena_create(size_t bytes, int flags, void **host, void **dev);
+hfq_status hfq_host_arena_destroy(void *host);
+
+/*
+ * Expert placement [PLACE] (host only, no allocation).
+ *   counts:   uint32 [L][E] calibration selection counts (decode heat).
+ *   resident_layers: N >= 0 keeps layers 0..N-1 fully in HBM; -1 = auto:
+ *            the largest N for which N full layers plus the hot sets of the
+ *            other L-N layers fit hbm_budget.
+ *   hot_per_layer: h >= 0; in every host layer its h most selected experts
+ *            (ties to the lower index) are placed in HBM too.
+ *   loc_out:  uint8 [L][E] out: 0 = HBM, 1 = host.
+ *   slot_out: int64 [L][E] out: index of the expert within its location's
+ *            arena, numbered in (layer, expert) order.
+ *   hbm_needed, host_needed: out, bytes per location.
+ * Returns HFQ_ERR_NOFIT, with the deficit in the message and both byte
+ * counts filled in, when the HBM part exceeds hbm_budget (loud refusal).
+ */
+hfq_status hfq_placement_build(int L, int E, size_t expert_bytes, const uint32_t *counts,
+                               int resident_layers, int hot_per_layer, size_t hbm_budget,
+                               uint8_t *loc_out, int64_t *slot_out, size_t *hbm_needed,
+                               size_t *host_needed);
+
+/*
+ * Pointer table from a placement (host only): out[l*E + e] = base + slot *
+ * expert_bytes with base = hbm_base for loc 0 and host_dev_base for loc 1.
+ */
+hfq_status hfq_placement_pointers(int L, int E, size_t expert_bytes, const uint8_t *loc,
+                                  const int64_t *slot, const void *hbm_base,
+                                  const void *host_dev_base, uint64_t *out);
+
+/*
+ * Read-bandwidth probe: a streaming kernel that reads `bytes` from `src`
+ * (HBM or host-mapped) `iters` times with 16-byte loads and writes one
+ * checksum word to `sink` (device).  Time it with events on `stream`.
+ */
+hfq_status hfq_probe_read(const void *src, size_t bytes, int iters, uint64_t *sink, void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* HFQ4MOE_H */

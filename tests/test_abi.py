@@ -1,0 +1,122 @@
+"""The C ABI without a GPU: the library loads, exports every function that
+include/*.h declares, and its host-only parts (sizes, host packer, placement,
+argument checks) agree with the oracle.  No call here launches a kernel."""
+import glob
+import os
+import re
+
+import numpy as np
+import pytest
+
+import expert_offload_b200 as eo
+from oracle import hfq4, placement
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared_functions():
+    names = set()
+    for h in glob.glob(os.path.join(ROOT, "include", "*.h")):
+        text = open(h).read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        for m in re.finditer(r"^[A-Za-z_][\w\s\*]*?\b([a-z_][a-z0-9_]*)\s*\(", text, flags=re.M):
+            line = m.group(0)
+            if line.startswith(("typedef", "#")):
+                continue
+            names.add(m.group(1))
+    return names
+
+
+@pytest.fixture(scope="module", autouse=True)
+def built():
+    from expert_offload_b200 import build
+    build.build()
+
+
+def test_every_declared_symbol_is_exported_and_bound():
+    declared = _declared_functions()
+    assert len(declared) >= 18
+    lib = eo.lib()
+    for name in declared:
+        assert hasattr(lib, name), name
+    assert declared == set(eo.symbols())
+
+
+def test_sizes_match_oracle():
+    for r, c in [(512, 2048), (2048, 512), (128, 256), (256, 128), (3, 300)]:
+        assert eo.hfq4_matrix_bytes(r, c) == hfq4.matrix_bytes(r, c)
+    for H, I in [(2048, 512), (256, 128), (384, 640)]:
+        assert eo.hfq4_expert_bytes(H, I) == hfq4.expert_bytes(H, I)
+    assert eo.hfq4_matrix_bytes(0, 5) == 0
+    assert eo.lib().hfq_version() >= 10000
+
+
+@pytest.mark.parametrize("E,H,I", [(2, 256, 128), (1, 512, 256), (3, 384, 640)])
+def test_host_pack_is_bit_identical_to_oracle(E, H, I):
+    rng = np.random.default_rng(E * H + I)
+    g = (rng.standard_normal((E, I, H)) * 0.02).astype(np.float32)
+    u = (rng.standard_normal((E, I, H)) * 0.02).astype(np.float32)
+    d = (rng.standard_normal((E, H, I)) * 0.02).astype(np.float32)
+    g[0, 0, :] = 0.5                       # a constant row (scale 0)
+    g[0, 1, :256] = np.float32(-0.25) + np.float32(0.0625) * (np.arange(256) % 16)   # exact grid
+    eb = hfq4.expert_bytes(H, I)
+    out = np.zeros(E * eb, dtype=np.uint8)
+    eo.hfq4_pack_experts(g, u, d, out, E, H, I)
+    ref = np.concatenate([hfq4.pack_expert(g[e], u[e], d[e]) for e in range(E)])
+    np.testing.assert_array_equal(out, ref)
+
+
+def test_host_pack_rejects_small_output():
+    g = np.zeros((1, 128, 256), np.float32)
+    out = np.zeros(10, np.uint8)
+    with pytest.raises(eo.HfqError) as e:
+        eo.hfq4_pack_experts(g, g, g.transpose(0, 2, 1).copy(), out, 1, 256, 128)
+    assert e.value.status == -1 and "needed" in e.value.message
+
+
+@pytest.mark.parametrize("N,h", [(0, 0), (2, 0), (1, 2), (-1, 3), (-1, 0), (4, 1)])
+def test_placement_matches_oracle(N, h):
+    rng = np.random.default_rng(N * 10 + h + 100)
+    counts = rng.integers(0, 20, (4, 9)).astype(np.uint32)
+    counts[1, 3] = counts[1, 5] = counts[1].max() + 1      # a tie in the hot ranking
+    eb = 1000
+    budget = 17_500
+    ref = placement.place(counts, eb, N, h, budget)
+    if ref.ok:
+        loc, slot, hn, hs = eo.hfq_placement_build(counts, eb, N, h, budget)
+        np.testing.assert_array_equal(loc, ref.loc)
+        np.testing.assert_array_equal(slot, ref.slot)
+        assert (hn, hs) == (ref.hbm_needed, ref.host_needed)
+    else:
+        with pytest.raises(eo.HfqError) as e:
+            eo.hfq_placement_build(counts, eb, N, h, budget)
+        assert e.value.status == -4
+        assert "DOES NOT FIT" in e.value.message and f"deficit {ref.deficit}" in e.value.message
+        assert e.value.hbm_needed == ref.hbm_needed
+
+
+def test_placement_pointers():
+    loc = np.array([[0, 1], [1, 0]], np.uint8)
+    slot = np.array([[0, 0], [1, 1]], np.int64)
+    p = eo.hfq_placement_pointers(loc, slot, 100, 0x10000, 0x90000)
+    assert p.tolist() == [[0x10000, 0x90000], [0x90000 + 100, 0x10000 + 100]]
+
+
+def test_argument_errors_are_caught_before_launch():
+    lib = eo.lib()
+    assert lib.moe_route(None, 1, 16, 4, None, None, None, None, None, None, 0, None) == -1
+    assert lib.moe_route(1024, 1, 600, 4, 1024, 1024, None, None, None, None, 0, None) == -3
+    assert lib.moe_route(1024, 1, 16, 17, 1024, 1024, None, None, None, None, 0, None) == -3
+    assert lib.moe_route(1024, 4, 16, 4, 1024, 1024, 1024, None, None, None, 0, None) == -1
+    assert lib.moe_route(1024, 4096, 16, 4, 1024, 1024, 1024, 1024, 1024, None, 0, None) == -8
+    lay = eo.Layer(1024, 16, 256, 100)                          # inter not a multiple of 128
+    assert lib.hfq4_moe_forward(eo.ctypes.byref(lay.struct), 1024, 0, 1, 1024, 1024, 4, None,
+                                None, None, 1024, None, 0, 1024, 1 << 20, None) == -3
+    lay = eo.Layer(1024, 16, 256, 128)
+    assert lib.hfq4_moe_forward(eo.ctypes.byref(lay.struct), 1024, 0, 1, 1024, 1024, 4, None,
+                                None, None, 1024, None, 0, 1024, 16, None) == -8   # workspace
+    assert lib.hfq4_moe_forward(eo.ctypes.byref(lay.struct), 1028, 0, 1, 1024, 1024, 4, None,
+                                None, None, 1024, None, 0, 1024, 1 << 20, None) == -2  # align
+    assert "16-byte" in eo.last_error()
+    assert lib.hfq4_dequant(1028, 1, 256, 1024, None) == -2
+    assert lib.hfq_host_arena_destroy(12345) == -1
