@@ -36,11 +36,17 @@ def parse():
     ap.add_argument("--steps", type=int, default=10000)
     ap.add_argument("--warmup", type=int, default=50)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=["decode"], default="decode")
+    ap.add_argument("--workload", choices=["decode", "verify", "offload"], default="decode")
+    ap.add_argument("--tokens", type=int, default=8, help="tokens per step (verify)")
+    ap.add_argument("--resident-layers", type=int, default=None, help="offload: N")
+    ap.add_argument("--hot", type=int, default=0, help="offload: hot experts per host layer")
+    ap.add_argument("--hbm-read-probe", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=2000)
     ap.add_argument("--distinct-tokens", type=int, default=64)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--path", type=int, default=0, help="0 auto, 1 GEMV")
+    ap.add_argument("--layers", type=int, default=None,
+                    help="a prefix of the stack (small profiling cases)")
     return ap.parse_args()
 
 
@@ -103,29 +109,92 @@ class ClockSampler:
 
 # ------------------------------------------------------------- our arm
 
-def build_decode(torch, w, G):
-    import numpy as np
+def workload_for(args):
+    """The workload a run measures (decode by default)."""
+    import dataclasses
 
-    import expert_offload_b200 as eo
-    from expert_offload_b200.model import ExpertStore
-    import synth
     from synth import workloads as W
+    w = W.WORKLOADS[{"decode": 2, "verify": 3, "offload": 5}[args.workload]]
+    if args.layers:
+        w = dataclasses.replace(w, layers=args.layers,
+                                name=f"{w.name} (first {args.layers} layers)")
+    T = args.tokens if args.workload == "verify" else 1
+    return w, T
 
-    def fill(l, g, u, d):
-        s = torch.cuda.current_stream().cuda_stream
-        E = g.shape[0]
-        synth.weights_dev(g.data_ptr(), w.seed, l, 0, E, synth.MAT_GATE, w.inter, w.hidden,
-                          W.WEIGHT_SIGMA, s)
-        synth.weights_dev(u.data_ptr(), w.seed, l, 0, E, synth.MAT_UP, w.inter, w.hidden,
-                          W.WEIGHT_SIGMA, s)
-        synth.weights_dev(d.data_ptr(), w.seed, l, 0, E, synth.MAT_DOWN, w.hidden, w.inter,
-                          W.WEIGHT_SIGMA, s)
 
-    store = ExpertStore(torch, w.layers, w.experts, w.hidden, w.inter, fill)
-    T = 1
-    logits = np.stack([W.logits_stack(w, g * T, T) for g in range(G)])          # [G, L, T, E]
-    xs = np.stack([W.activations(w, g * T, T)[0] for g in range(G)])            # [G, T, H] bf16
-    return eo, store, logits, xs
+def placement_for(eo, args, w):
+    """Location/slot tables: all resident, or the offload split."""
+    if args.workload != "offload":
+        return None, None, None
+    from synth import workloads as W
+    counts = W.calibration_counts(w, 1024)
+    eb = eo.hfq4_expert_bytes(w.hidden, w.inter)
+    N = w.layers if args.resident_layers is None else args.resident_layers
+    loc, slot, hn, hs = eo.hfq_placement_build(counts, eb, N, args.hot, 170 * 2**30)
+    return loc, slot, {"resident_layers": N, "hot_per_layer": args.hot, "hbm_bytes": hn,
+                       "host_bytes": hs}
+
+
+def step_bytes(logits_g, k, eb, loc):
+    """(HBM bytes, host bytes) one step streams: every unique selected expert of
+    every layer once (router logits and activations, < 0.1 %, not counted)."""
+    import numpy as np
+    hbm = host = 0
+    for l in range(logits_g.shape[0]):
+        top = np.argpartition(-logits_g[l], k - 1, axis=1)[:, :k]
+        for e in np.unique(top):
+            if loc is not None and loc[l, e]:
+                host += eb
+            else:
+                hbm += eb
+    return hbm, host
+
+
+def measure_pcie(torch, eo, nbytes=1 << 30):
+    """Host-to-device bandwidth two ways: a pinned cudaMemcpy and the zero-copy
+    read kernel over a mapped arena (the strata report's link probe, done here
+    with the expert kernel's own load path)."""
+    h, d = eo.hfq_host_arena_create(nbytes)
+    try:
+        sink = torch.zeros(1, dtype=torch.int64, device="cuda")
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        eo.hfq_probe_read(d, nbytes, 1, sink)
+        torch.cuda.synchronize()
+        e0.record()
+        eo.hfq_probe_read(d, nbytes, 2, sink)
+        e1.record()
+        torch.cuda.synchronize()
+        zc = 2 * nbytes / (e0.elapsed_time(e1) / 1e3) / 1e9
+        import ctypes
+
+        import numpy as np
+        buf = (ctypes.c_uint8 * nbytes).from_address(h)
+        src = torch.from_numpy(np.frombuffer(buf, dtype=np.uint8))
+        dst = torch.empty(nbytes, dtype=torch.uint8, device="cuda")
+        dst.copy_(src, non_blocking=True)
+        torch.cuda.synchronize()
+        e0.record()
+        dst.copy_(src, non_blocking=True)
+        e1.record()
+        torch.cuda.synchronize()
+        cp = nbytes / (e0.elapsed_time(e1) / 1e3) / 1e9
+    finally:
+        eo.hfq_host_arena_destroy(h)
+    return {"zero_copy_read_gbs": round(zc, 2), "pinned_memcpy_gbs": round(cp, 2)}
+
+
+def measure_hbm_read(torch, eo, nbytes=4 << 30):
+    sink = torch.zeros(1, dtype=torch.int64, device="cuda")
+    buf = torch.empty(nbytes, dtype=torch.uint8, device="cuda")
+    eo.hfq_probe_read(buf, nbytes, 1, sink)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    e0.record()
+    eo.hfq_probe_read(buf, nbytes, 3, sink)
+    e1.record()
+    torch.cuda.synchronize()
+    del buf
+    return round(3 * nbytes / (e0.elapsed_time(e1) / 1e3) / 1e9, 1)
 
 
 def run_ours(args, rank, world, local_rank):
@@ -140,13 +209,28 @@ def run_ours(args, rank, world, local_rank):
         import torch.distributed as dist
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=torch.device("cuda", local_rank))
+    import expert_offload_b200 as eo
+    import synth
+    from expert_offload_b200.model import ExpertStore
     from synth import workloads as W
 
-    w = W.WORKLOADS[2]
-    G = args.distinct_tokens
-    eo, store, logits, xs = build_decode(torch, w, G)
-    L, H, I, E, k, T = w.layers, w.hidden, w.inter, w.experts, w.top_k, 1
+    w, T = workload_for(args)
+    L, H, I, E, k = w.layers, w.hidden, w.inter, w.experts, w.top_k
     eb = eo.hfq4_expert_bytes(H, I)
+    G = args.distinct_tokens
+    loc, slot, place_info = placement_for(eo, args, w)
+
+    def fill(l, g, u, d):
+        s = torch.cuda.current_stream().cuda_stream
+        synth.weights_dev(g.data_ptr(), w.seed, l, 0, E, synth.MAT_GATE, I, H, W.WEIGHT_SIGMA, s)
+        synth.weights_dev(u.data_ptr(), w.seed, l, 0, E, synth.MAT_UP, I, H, W.WEIGHT_SIGMA, s)
+        synth.weights_dev(d.data_ptr(), w.seed, l, 0, E, synth.MAT_DOWN, H, I, W.WEIGHT_SIGMA, s)
+
+    store = ExpertStore(torch, L, E, H, I, fill, loc=loc, slot=slot)
+    logits = np.stack([np.stack([W.logits(w, l, g * T, T) for l in range(L)])
+                       for g in range(G)])                                       # [G, L, T, E]
+    xs = np.stack([W.activations(w, g * T, T)[0] for g in range(G)])            # [G, T, H] bf16
+    per_group = [step_bytes(logits[g], k, eb, loc) for g in range(G)]
     d_logits = torch.from_numpy(logits).cuda()
     d_x = torch.from_numpy(xs.view(np.int16)).cuda()
     x_out = torch.empty((G, T, H), dtype=torch.int16, device="cuda")
@@ -159,24 +243,32 @@ def run_ours(args, rank, world, local_rank):
         eo.hfq4_moe_decode_stack(store.layers, d_logits[g], k, d_x[g], T, x_out[g], ws,
                                  path=args.path, stream=s, _layer_array=arr)
 
-    # graphs: one per distinct token (the persistent path is one launch per step
-    # either way; graphs remove host launch cost from the device timeline)
     with torch.cuda.stream(stream):
         for g in range(G):
             step(g, stream)
     torch.cuda.synchronize()
+    eo.hfq_workspace_status(ws, stream)
     graphs = []
-    for g in range(G):
-        gr = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(gr, stream=stream):
-            step(g, stream)
-        graphs.append(gr)
-    torch.cuda.synchronize()
-    launches_per_step = eo_launches_per_step(eo, L)
+    try:
+        for g in range(G):
+            gr = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(gr, stream=stream):
+                step(g, stream)
+            graphs.append(gr)
+        torch.cuda.synchronize()
+        replay = [gr.replay for gr in graphs]
+        launch_mode = "cuda graph per token group"
+    except RuntimeError as exc:          # capture not possible: launch directly
+        print(f"graph capture failed ({exc}); launching directly", file=sys.stderr)
+        torch.cuda.synchronize()
+        graphs = []
+        replay = [(lambda g=g: step(g, stream)) for g in range(G)]
+        launch_mode = "direct launch"
+    launches_per_step = eo.hfq4_stack_launches(L, T, k, H, I)
 
     with torch.cuda.stream(stream):
         for i in range(args.warmup):
-            graphs[i % G].replay()
+            replay[i % G]()
     torch.cuda.synchronize()
     if dist:
         dist.barrier()
@@ -190,7 +282,7 @@ def run_ours(args, rank, world, local_rank):
     with torch.cuda.stream(stream):
         ev[0].record(stream)
         for i in range(K):
-            graphs[i % G].replay()
+            replay[i % G]()
             ev[i + 1].record(stream)
     torch.cuda.synchronize()
     if dist:
@@ -209,36 +301,37 @@ def run_ours(args, rank, world, local_rank):
     in_x = torch.empty_like(d_x[0])
     out_x = torch.empty_like(x_out[0])
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+
+    def e2e_step(i):
+        g = i % G
+        in_l.copy_(h_logits[g], non_blocking=True)
+        in_x.copy_(h_x[g], non_blocking=True)
+        eo.hfq4_moe_decode_stack(store.layers, in_l, k, in_x, T, out_x, ws, path=args.path,
+                                 stream=stream, _layer_array=arr)
+        h_out[g].copy_(out_x, non_blocking=True)
+
     with torch.cuda.stream(stream):
         for i in range(min(20, K2)):
-            g = i % G
-            in_l.copy_(h_logits[g], non_blocking=True)
-            in_x.copy_(h_x[g], non_blocking=True)
-            eo.hfq4_moe_decode_stack(store.layers, in_l, k, in_x, T, out_x, ws, path=args.path,
-                                     stream=stream, _layer_array=arr)
-            h_out[g].copy_(out_x, non_blocking=True)
+            e2e_step(i)
         torch.cuda.synchronize()
         e0.record(stream)
         for i in range(K2):
-            g = i % G
-            in_l.copy_(h_logits[g], non_blocking=True)
-            in_x.copy_(h_x[g], non_blocking=True)
-            eo.hfq4_moe_decode_stack(store.layers, in_l, k, in_x, T, out_x, ws, path=args.path,
-                                     stream=stream, _layer_array=arr)
-            h_out[g].copy_(out_x, non_blocking=True)
+            e2e_step(i)
         e1.record(stream)
     torch.cuda.synchronize()
     e2e_ms = e0.elapsed_time(e1)
+    eo.hfq_workspace_status(ws, stream)
 
     if dist:
         t = torch.tensor([total_ms, e2e_ms], dtype=torch.float64, device="cuda")
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         total_ms, e2e_ms = float(t[0]), float(t[1])
 
-    bytes_per_step = L * k * eb * T      # T = 1: k unique experts per layer
+    hbm_b = sum(per_group[i % G][0] for i in range(K)) / K
+    host_b = sum(per_group[i % G][1] for i in range(K)) / K
+    bytes_per_step = hbm_b + host_b
     value = world * K * T / (total_ms / 1e3)
     mean_launch_ms = sum(per_launch) / K
-    achieved = bytes_per_step / (mean_launch_ms / 1e3) / 1e9
     peak, peak_kind = peaks()
     out = {
         "metric": METRIC, "value": round(value, 2), "unit": "tokens/s", "n_gpus": world,
@@ -248,22 +341,52 @@ def run_ours(args, rank, world, local_rank):
         "config": {"workload": w.name, "layers": L, "hidden": H, "inter": I, "experts": E,
                    "top_k": k, "tokens_per_step": T, "weights": "hfq4 (136-byte blocks)",
                    "activations": "bf16", "accumulate": "f32",
-                   "distinct_tokens_cycled": G, "bytes_per_step": bytes_per_step,
-                   "l2": "per-step working set 535 MB > 126 MB L2, no flush",
+                   "distinct_token_groups_cycled": G,
+                   "expert_bytes_per_step": round(bytes_per_step),
+                   "launch": launch_mode,
+                   "l2": "per-step working set > 126 MB L2 (every step routes new tokens); "
+                         "no flush",
                    "parallelism": f"replicas x{world}"},
-        "achieved_gbs": round(bytes_per_step * world * K / (total_ms / 1e3) / 1e9, 1),
-        "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak,
-                     "unit": "GB/s", "frac": round(achieved / peak, 4), "traffic": None,
-                     "peak_source": peak_kind,
-                     "kernel": "decode stack step (one launch sequence per token)",
-                     "bytes_per_launch": bytes_per_step,
-                     "mean_launch_ms": round(mean_launch_ms, 5)},
-        "e2e": {"value": round(world * K2 * T / (e2e_ms / 1e3), 2), "unit": "tokens/s",
-                "h2d_bytes_per_step": int(in_l.numel() * 4 + in_x.numel() * 2),
-                "d2h_bytes_per_step": int(out_x.numel() * 2)},
         "gpu_launches": launches_per_step * K,
         "clocks": clocks,
     }
+    kernel = ("stack_kernel (persistent: all layers of one step per launch)"
+              if launches_per_step == 1 else "per-layer route + gate/up + down launches")
+    if args.workload == "offload":
+        pcie = measure_pcie(torch, eo)
+        bw_pcie = max(pcie.values())
+        roof_ms = 0.0
+        for g in range(G):
+            # per layer the HBM and PCIe streams overlap: max of the two, summed
+            lg = logits[g]
+            for l in range(L):
+                hb, hs = step_bytes(lg[l:l + 1], k, eb, loc[l:l + 1])
+                roof_ms += max(hb / (peak * 1e9), hs / (bw_pcie * 1e9)) * 1e3
+        roof_ms /= G
+        out["config"]["placement"] = place_info
+        out["config"]["pcie"] = pcie
+        out["roofline"] = {"bound": "pcie" if host_b > 0 else "hbm",
+                           "achieved": round(bytes_per_step / (mean_launch_ms / 1e3) / 1e9, 2),
+                           "peak": round(bytes_per_step / (roof_ms / 1e3) / 1e9, 2),
+                           "unit": "GB/s", "frac": round(roof_ms / mean_launch_ms, 4),
+                           "traffic": None, "kernel": kernel,
+                           "peak_source": f"roofline time from measured PCIe {bw_pcie} GB/s "
+                                          f"and {peak_kind} HBM {peak} GB/s per layer",
+                           "hbm_bytes_per_launch": round(hbm_b),
+                           "host_bytes_per_launch": round(host_b),
+                           "mean_launch_ms": round(mean_launch_ms, 5)}
+    else:
+        achieved = bytes_per_step / (mean_launch_ms / 1e3) / 1e9
+        out["roofline"] = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak,
+                           "unit": "GB/s", "frac": round(achieved / peak, 4), "traffic": None,
+                           "peak_source": peak_kind, "kernel": kernel,
+                           "bytes_per_launch": round(bytes_per_step),
+                           "mean_launch_ms": round(mean_launch_ms, 5)}
+        if args.hbm_read_probe:
+            out["roofline"]["hbm_read_probe_gbs"] = measure_hbm_read(torch, eo)
+    out["e2e"] = {"value": round(world * K2 * T / (e2e_ms / 1e3), 2), "unit": "tokens/s",
+                  "h2d_bytes_per_step": int(in_l.numel() * 4 + in_x.numel() * 2),
+                  "d2h_bytes_per_step": int(out_x.numel() * 2)}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         out["cpu_baseline"] = cpu_baseline(w)
     if dist:
@@ -272,11 +395,6 @@ def run_ours(args, rank, world, local_rank):
         dist.destroy_process_group()
     store.close()
     return out
-
-
-def eo_launches_per_step(eo, L):
-    # route + gate/up + down per layer for the per-layer path
-    return 3 * L
 
 
 # ------------------------------------------------------- oracle (CPU) arms

@@ -58,9 +58,11 @@ _SIGS = {
     "hfq4_moe_forward": (_i, [ctypes.POINTER(hfq4_layer), _vp, _i, _i, _vp, _vp, _i, _vp, _vp,
                               _vp, _vp, _vp, _i, _vp, _sz, _vp]),
     "hfq4_stack_workspace_bytes": (_sz, [_i, _i, _i, _i, _i]),
+    "hfq4_stack_launches": (_i, [_i, _i, _i, _i, _i]),
     "hfq4_moe_decode_stack": (_i, [ctypes.POINTER(hfq4_layer), _i, _vp, _i, _vp, _i, _vp, _vp,
                                    _vp, _vp, _i, _vp, _sz, _vp]),
     "hfq_workspace_status": (_i, [_vp, _sz, _vp]),
+    "hfq_set_option": (_i, [_i, ctypes.c_longlong]),
     "hfq_host_arena_create": (_i, [_sz, _i, ctypes.POINTER(_vp), ctypes.POINTER(_vp)]),
     "hfq_host_arena_destroy": (_i, [_vp]),
     "hfq_placement_build": (_i, [_i, _i, _sz, _vp, _i, _i, _sz, _vp, _vp,
@@ -198,6 +200,10 @@ def hfq4_stack_workspace_bytes(T: int, k: int, hidden: int, inter: int, n_expert
     return lib().hfq4_stack_workspace_bytes(T, k, hidden, inter, n_experts)
 
 
+def hfq4_stack_launches(n_layers: int, T: int, k: int, hidden: int, inter: int) -> int:
+    return lib().hfq4_stack_launches(n_layers, T, k, hidden, inter)
+
+
 def layer_array(layers):
     arr = (hfq4_layer * len(layers))()
     for i, l in enumerate(layers):
@@ -212,6 +218,13 @@ def hfq4_moe_decode_stack(layers, logits, k: int, x0, T: int, x_out, workspace, 
     _check(lib().hfq4_moe_decode_stack(arr, len(layers), _ptr(logits), k, _ptr(x0), T, _ptr(x_out),
                                        _ptr(y_all), _ptr(idx_all), _ptr(wts_all), path,
                                        _ptr(workspace), _nbytes(workspace), _stream(stream)))
+
+
+OPT_WAIT_TIMEOUT_NS, OPT_TEST_MISSING_ARRIVALS, OPT_TIMELINE_BUFFER = 1, 2, 3
+
+
+def hfq_set_option(option: int, value: int) -> None:
+    _check(lib().hfq_set_option(option, value))
 
 
 def hfq_workspace_status(workspace, stream=None) -> None:

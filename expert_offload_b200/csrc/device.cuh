@@ -49,4 +49,18 @@ constexpr size_t kWsHeader = sizeof(WsHeader);   // 256 bytes
 
 inline cudaError_t launch_check() { return cudaGetLastError(); }
 
+// Persistent decode kernel (stack.cu).
+bool stack_supported(int T, int H, int I, int k, int G);
+size_t stack_ctl_bytes();
+hfq_status launch_stack(const hfq4_layer *layers, int L, const float *logits, const int32_t *idx_in,
+                        const float *wts_in, const void *x0, bool x0_f32, int T, int k,
+                        uint16_t *x_out, uint16_t *xbuf, float *h, float *y, uint16_t *y_bf16,
+                        int32_t *idx_all, float *wts_all, unsigned *ctl, long long timeout_ns,
+                        int extra_arrivals, cudaStream_t s);
+
+// Library options (hfq_set_option).
+long long option_wait_timeout_ns();
+int option_take_extra_arrivals();     // one-shot test hook
+void *option_timeline();              // debug: device buffer for phase stamps, or null
+
 }  // namespace hfq

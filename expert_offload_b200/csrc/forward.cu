@@ -160,6 +160,18 @@ size_t h_bytes(int T, int k, int I)
 
 size_t act_bytes(int T, int H) { return ((size_t)T * H * 2 + 255) / 256 * 256; }
 
+int num_sms_fwd()
+{
+    static int n = 0;
+    if (!n) {
+        int dev = 0;
+        cudaGetDevice(&dev);
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+        if (n <= 0) n = 148;
+    }
+    return n;
+}
+
 hfq_status check_ws(void *ws, size_t ws_bytes, size_t need)
 {
     if (!ws || ws_bytes < need)
@@ -204,14 +216,48 @@ hfq_status check_layer(const hfq4_layer *layer, int k)
 }  // namespace
 }  // namespace hfq
 
+namespace hfq {
+static long long g_timeout_ns = 1000000000LL;   // 1 s per bounded wait
+static int g_extra_arrivals = 0;
+static void *g_timeline = nullptr;
+void *option_timeline() { return g_timeline; }
+long long option_wait_timeout_ns() { return g_timeout_ns; }
+int option_take_extra_arrivals()
+{
+    int v = g_extra_arrivals;
+    g_extra_arrivals = 0;
+    return v;
+}
+}  // namespace hfq
+
 using namespace hfq;
 
 extern "C" {
 
+hfq_status hfq_set_option(int option, long long value)
+{
+    switch (option) {
+    case HFQ_OPT_WAIT_TIMEOUT_NS:
+        if (value < 1000 || value > 60000000000LL)
+            return fail(HFQ_ERR_ARG, "wait timeout %lld ns outside [1 us, 60 s]", value);
+        g_timeout_ns = value;
+        return ok();
+    case HFQ_OPT_TEST_MISSING_ARRIVALS:
+        if (value < 0 || value > 1024) return fail(HFQ_ERR_ARG, "bad value %lld", value);
+        g_extra_arrivals = (int)value;
+        return ok();
+    case HFQ_OPT_TIMELINE_BUFFER:
+        g_timeline = reinterpret_cast<void *>((uintptr_t)value);
+        return ok();
+    default:
+        return fail(HFQ_ERR_ARG, "unknown option %d", option);
+    }
+}
+
 size_t hfq4_moe_workspace_bytes(int T, int k, int hidden, int inter, int n_experts)
 {
     if (T < 1 || k < 1 || hidden < 1 || inter < 1 || n_experts < 1) return 0;
-    return kWsHeader + h_bytes(T, k, inter);
+    return stack_ctl_bytes() + h_bytes(T, k, inter);
 }
 
 hfq_status hfq4_moe_forward(const hfq4_layer *layer, const void *x, hfq_dtype x_dtype, int T,
@@ -231,17 +277,30 @@ hfq_status hfq4_moe_forward(const hfq4_layer *layer, const void *x, hfq_dtype x_
         return fail(HFQ_ERR_ALIGN, "x, y and y_bf16 must be 16-byte aligned");
     size_t need = hfq4_moe_workspace_bytes(T, k, layer->hidden, layer->inter, layer->n_experts);
     if ((st = check_ws(workspace, ws_bytes, need))) return st;
-    float *h = reinterpret_cast<float *>(static_cast<char *>(workspace) + kWsHeader);
-    st = launch_layer(*layer, x, x_dtype, T, idx, wts, k, y, y_bf16, h, nullptr, nullptr,
-                      (cudaStream_t)stream);
+    float *h = reinterpret_cast<float *>(static_cast<char *>(workspace) + stack_ctl_bytes());
+    if (stack_supported(T, layer->hidden, layer->inter, k, num_sms_fwd())) {
+        st = launch_stack(layer, 1, nullptr, idx, wts, x, x_dtype == HFQ_F32, T, k, nullptr,
+                          nullptr, h, y, static_cast<uint16_t *>(y_bf16), nullptr, nullptr,
+                          static_cast<unsigned *>(workspace), option_wait_timeout_ns(),
+                          option_take_extra_arrivals(), (cudaStream_t)stream);
+    } else {
+        st = launch_layer(*layer, x, x_dtype, T, idx, wts, k, y, y_bf16, h, nullptr, nullptr,
+                          (cudaStream_t)stream);
+    }
     return st ? st : ok();
 }
 
 size_t hfq4_stack_workspace_bytes(int T, int k, int hidden, int inter, int n_experts)
 {
     if (T < 1 || T > 8 || k < 1 || hidden < 1 || inter < 1 || n_experts < 1) return 0;
-    return kWsHeader + h_bytes(T, k, inter) + 2 * act_bytes(T, hidden) +
+    return stack_ctl_bytes() + h_bytes(T, k, inter) + 2 * act_bytes(T, hidden) +
            ((size_t)T * k * 8 + 255) / 256 * 256;
+}
+
+int hfq4_stack_launches(int n_layers, int T, int k, int hidden, int inter)
+{
+    if (n_layers < 1 || n_layers > HFQ_MAX_STACK_LAYERS || T < 1 || T > 8 || k < 1) return 0;
+    return stack_supported(T, hidden, inter, k, num_sms_fwd()) ? 1 : 3 * n_layers;
 }
 
 hfq_status hfq4_moe_decode_stack(const hfq4_layer *layers, int n_layers, const float *logits,
@@ -269,7 +328,7 @@ hfq_status hfq4_moe_decode_stack(const hfq4_layer *layers, int n_layers, const f
     const int H = layers[0].hidden, I = layers[0].inter, E = layers[0].n_experts;
     size_t need = hfq4_stack_workspace_bytes(T, k, H, I, E);
     if ((st = check_ws(workspace, ws_bytes, need))) return st;
-    char *ws = static_cast<char *>(workspace) + kWsHeader;
+    char *ws = static_cast<char *>(workspace) + stack_ctl_bytes();
     float *h = reinterpret_cast<float *>(ws);
     ws += h_bytes(T, k, I);
     uint16_t *xa = reinterpret_cast<uint16_t *>(ws);
@@ -279,6 +338,13 @@ hfq_status hfq4_moe_decode_stack(const hfq4_layer *layers, int n_layers, const f
     int32_t *idx = reinterpret_cast<int32_t *>(ws);
     float *wts = reinterpret_cast<float *>(ws + (size_t)T * k * 4);
     cudaStream_t s = (cudaStream_t)stream;
+    if (stack_supported(T, H, I, k, num_sms_fwd())) {
+        st = launch_stack(layers, n_layers, logits, nullptr, nullptr, x0, false, T, k,
+                          static_cast<uint16_t *>(x_out), xa, h, y_all, nullptr, idx_all, wts_all,
+                          static_cast<unsigned *>(workspace), option_wait_timeout_ns(),
+                          option_take_extra_arrivals(), s);
+        return st ? st : ok();
+    }
     const uint16_t *cur = static_cast<const uint16_t *>(x0);
     for (int l = 0; l < n_layers; ++l) {
         uint16_t *next = (l == n_layers - 1) ? static_cast<uint16_t *>(x_out) : (l & 1 ? xb : xa);
@@ -302,8 +368,9 @@ hfq_status hfq_workspace_status(void *workspace, size_t ws_bytes, void *stream)
     if (err == cudaSuccess) err = cudaStreamSynchronize(s);
     if (err != cudaSuccess) return fail(HFQ_ERR_CUDA, "status read: %s", cudaGetErrorString(err));
     if (word != 0) {
-        unsigned int zero = 0;
-        cudaMemcpyAsync(workspace, &zero, sizeof zero, cudaMemcpyHostToDevice, s);
+        // the wound-down launch left its counters behind: clear the whole control block
+        size_t n = ws_bytes < stack_ctl_bytes() ? ws_bytes : stack_ctl_bytes();
+        cudaMemsetAsync(workspace, 0, n, s);
         cudaStreamSynchronize(s);
         return fail((hfq_status)(int)word, "a device-side wait ran out (status %d)", (int)word);
     }

@@ -196,15 +196,41 @@ hfq_status hfq4_moe_forward(const hfq4_layer *layer, const void *x, hfq_dtype x_
  *   T <= 8.  workspace: hfq4_stack_workspace_bytes(T, k, H, I, E) bytes.
  */
 size_t hfq4_stack_workspace_bytes(int T, int k, int hidden, int inter, int n_experts);
+/* Kernel launches one hfq4_moe_decode_stack call makes (1 when the whole stack
+ * runs as one persistent launch, 3 per layer otherwise); 0 on bad arguments. */
+int hfq4_stack_launches(int n_layers, int T, int k, int hidden, int inter);
 hfq_status hfq4_moe_decode_stack(const hfq4_layer *layers, int n_layers, const float *logits,
                                  int k, const void *x0, int T, void *x_out, float *y_all,
                                  int32_t *idx_all, float *wts_all, int path, void *workspace,
                                  size_t ws_bytes, void *stream);
 
 /*
+ * Library options (process-wide, host side):
+ *   HFQ_OPT_WAIT_TIMEOUT_NS: deadline of every bounded device-side wait
+ *     (grid barriers, expert counters, ring barriers), default 1 s.  When a
+ *     wait runs out, the kernel records HFQ_ERR_TIMEOUT in the workspace
+ *     status word, stops doing work, lets its copies in flight land and exits.
+ *   HFQ_OPT_TEST_MISSING_ARRIVALS: fault injection for tests; the next
+ *     persistent-kernel launch makes its grid barriers wait for this many
+ *     CTAs that do not exist, so the wait runs out without any fault.
+ *   HFQ_OPT_TIMELINE_BUFFER: debug; the device address of a u64 buffer of
+ *     2 * n_layers * 32 words, zero-filled (0 = off).  Persistent-kernel
+ *     launches then write %globaltimer stamps (ns) for two CTAs (CTA 0 and CTA
+ *     gridDim/2), per layer: [0] layer start, [1] routed, [2] table built,
+ *     [3 + s] ring stage s ready (s < 12), [16] gate/up done, [17] all h
+ *     ready, [18] h staged, [19] down done, [20] layer end.
+ * Returns HFQ_ERR_ARG for an unknown option or a value out of range.
+ */
+#define HFQ_OPT_WAIT_TIMEOUT_NS 1
+#define HFQ_OPT_TEST_MISSING_ARRIVALS 2
+#define HFQ_OPT_TIMELINE_BUFFER 3
+hfq_status hfq_set_option(int option, long long value);
+
+/*
  * Device status word of a workspace (synchronises `stream`): HFQ_OK, or
  * HFQ_ERR_TIMEOUT if a bounded device-side wait of a previous call ran out.
- * The word is cleared by the read.
+ * After a timeout the word and the workspace's control block are cleared.
+ * A new workspace must be zero-filled before its first use.
  */
 hfq_status hfq_workspace_status(void *workspace, size_t ws_bytes, void *stream);
 

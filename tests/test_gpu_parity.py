@@ -170,9 +170,11 @@ def test_forward_tiny_workload_all_tokens(eo):
     ref = moe.moe_layer(oracle_layer, H, I, x.astype(np.float64), ridx, rw)
     err = max_rel_err(y.cpu().numpy(), ref)
     assert err <= TOL, err
-    # bf16 output: within one bf16 step of the oracle's value
-    yb32 = yb.float().cpu().numpy().astype(np.float64)
-    assert np.all(np.abs(yb32 - ref) <= np.abs(ref) * 2**-7 + 1e-30)
+    # bf16 output: the f32 result rounded once, so within half a bf16 step of
+    # a value that is itself within the f32 tolerance of the oracle
+    yb32 = yb.float().cpu().numpy().astype(np.float64).reshape(ref.shape)
+    bound = np.abs(ref) * 2**-8 + TOL * np.max(np.abs(ref), axis=1, keepdims=True)
+    assert np.all(np.abs(yb32 - ref) <= bound)
     assert_guards(raw, T * H * 4)
     assert_guards(rawb, T * H * 2)
 
@@ -216,16 +218,75 @@ def test_forward_decode_shape(eo, decode_layer, T):
 @pytest.mark.slow
 def test_decode_stack_full_workload(eo):
     """The 40-layer, 256-expert decode stack at T = 1, in the launch the bench
-    times, against the oracle's own residual chain."""
+    times.  A bf16 residual stream is not unique: where x_l + y_l lands within
+    rounding error of a bf16 midpoint, either neighbour is a correct result,
+    and two correct chains then differ from that layer on.  So the test pins
+    what is unique: (1) the routing of every layer (logits are inputs);
+    (2) every layer, run by the same persistent kernel on the oracle's own
+    x_l, against the oracle's y_l; (3) the chained launch on its leading
+    layers, and its final residual within 1e-2 relative L2 of the oracle's."""
     from expert_offload_b200.model import ExpertStore
     w = W.WORKLOADS[2]
     H, I, E, k, L, T = w.hidden, w.inter, w.experts, w.top_k, w.layers, 1
     store = ExpertStore(torch, L, E, H, I, device_fill(torch, w))
     logits = W.logits_stack(w, 0, T)                             # [L, T, E]
     x0, _ = W.activations(w, 0, T)
-    d_logits = torch.from_numpy(logits).cuda()
-    d_x0 = torch.from_numpy(x0.view(np.int16)).cuda()
-    x_out = torch.empty((T, H), dtype=torch.int16, device="cuda")
+    caches = [moe.ExpertCache(OraclePackedLayer(w, l), H, I) for l in range(L)]
+    ys, xs = moe.residual_stack(caches, logits, synth.bf16_bits_to_f32(x0).astype(np.float64), k,
+                                route.route)
+    # (1) + (3): the chained 40-layer launch
+    x_out, y_all, idx_all, _, _ = _run_stack(eo, store, logits, x0, k, T, H, E, L, I)
+    np.testing.assert_array_equal(idx_all.cpu().numpy(),
+                                  np.stack([route.route(logits[l], k)[0] for l in range(L)]))
+    y_gpu = y_all.cpu().numpy()
+    lead = [max_rel_err(y_gpu[l], ys[l]) for l in range(4)]
+    assert max(lead) <= TOL, lead
+    xg = synth.bf16_bits_to_f32(x_out.cpu().numpy().view(np.uint16)).astype(np.float64)
+    assert np.linalg.norm(xg - xs[-1]) <= 1e-2 * np.linalg.norm(xs[-1])
+    # (2): every layer in isolation on the oracle's input
+    for l in range(L):
+        xl = synth.to_bf16_bits(xs[l].astype(np.float32))
+        _, y1, _, _, _ = _run_stack(eo, _OneLayer(store, l), logits[l:l + 1], xl, k, T, H, E, 1, I)
+        err = max_rel_err(y1.cpu().numpy()[0], ys[l])
+        assert err <= TOL, (l, err)
+    # spot-check the device-packed bytes of some used experts
+    used = idx_all.cpu().numpy()
+    for l in (0, L // 2, L - 1):
+        e = int(used[l, 0, 0])
+        np.testing.assert_array_equal(store.expert_bytes_at(l, e), caches[l].experts[e])
+
+
+class _OneLayer:
+    """A view of one layer of a store, with the store's interface."""
+
+    def __init__(self, store, l):
+        self.layers = [store.layers[l]]
+
+
+def test_forward_per_layer_path_beyond_eight_tokens(eo):
+    """T = 16 runs the per-layer kernels (the persistent kernel takes T <= 8)."""
+    from expert_offload_b200.model import ExpertStore
+    w = W.WORKLOADS[1]
+    H, I, E, k, T = w.hidden, w.inter, w.experts, w.top_k, 16
+    store = ExpertStore(torch, 1, E, H, I, device_fill(torch, w))
+    logits = W.logits(w, 0, 0, T)
+    x, _ = W.activations(w, 0, T)
+    ridx, rw = route.route(logits, k)
+    idx, wts = _route_gpu(eo, logits, k, False)
+    raw, y = guarded(T * H, torch.float32)
+    wsb = ws(eo.hfq4_moe_workspace_bytes(T, k, H, I, E))
+    eo.hfq4_moe_forward(store.layers[0], torch.from_numpy(x).cuda(), eo.HFQ_F32, T,
+                        torch.from_numpy(idx).cuda(), torch.from_numpy(wts).cuda(), k, y, wsb)
+    torch.cuda.synchronize()
+    ref = moe.moe_layer(OraclePackedLayer(w, 0), H, I, x.astype(np.float64), ridx, rw)
+    assert max_rel_err(y.cpu().numpy(), ref) <= TOL
+    assert_guards(raw, T * H * 4)
+
+
+def _run_stack(eo, store, logits, x0_bits, k, T, H, E, L, I):
+    d_logits = torch.from_numpy(np.ascontiguousarray(logits)).cuda()
+    d_x0 = torch.from_numpy(x0_bits.view(np.int16)).cuda()
+    rawx, x_out = guarded(T * H, torch.int16)
     y_all = torch.empty((L, T, H), dtype=torch.float32, device="cuda")
     idx_all = torch.empty((L, T, k), dtype=torch.int32, device="cuda")
     wts_all = torch.empty((L, T, k), dtype=torch.float32, device="cuda")
@@ -234,21 +295,70 @@ def test_decode_stack_full_workload(eo):
                              idx_all=idx_all, wts_all=wts_all)
     torch.cuda.synchronize()
     eo.hfq_workspace_status(wsb)
+    assert_guards(rawx, T * H * 2)
+    return x_out, y_all, idx_all, wts_all, wsb
+
+
+@pytest.fixture(scope="module")
+def verify_model(eo):
+    """Three layers of the 512-expert verify workload (layers 0..2), resident."""
+    from expert_offload_b200.model import ExpertStore
+    w = W.WORKLOADS[3]
+    store = ExpertStore(torch, 3, w.experts, w.hidden, w.inter, device_fill(torch, w))
+    return w, store
+
+
+@pytest.mark.parametrize("T", [1, 2, 5, 8])
+def test_verify_stack_multi_token(eo, verify_model, T):
+    """The persistent kernel on speculative-verify batches (skewed routing,
+    512 experts): every layer's y against the oracle's residual chain."""
+    w, store = verify_model
+    H, I, E, k, L = w.hidden, w.inter, w.experts, w.top_k, 3
+    logits = np.stack([W.logits(w, l, 40 * T, T) for l in range(L)])
+    x0, _ = W.activations(w, 40 * T, T)
+    x_out, y_all, idx_all, wts_all, _ = _run_stack(eo, store, logits, x0, k, T, H, E, L, I)
     caches = [moe.ExpertCache(OraclePackedLayer(w, l), H, I) for l in range(L)]
     ys, xs = moe.residual_stack(caches, logits, synth.bf16_bits_to_f32(x0).astype(np.float64), k,
                                 route.route)
-    np.testing.assert_array_equal(idx_all.cpu().numpy(),
-                                  np.stack([route.route(logits[l], k)[0] for l in range(L)]))
-    y_gpu = y_all.cpu().numpy()
-    errs = [max_rel_err(y_gpu[l], ys[l]) for l in range(L)]
+    for l in range(L):
+        ridx, rw = route.route(logits[l], k)
+        np.testing.assert_array_equal(idx_all.cpu().numpy()[l], ridx)
+        np.testing.assert_allclose(wts_all.cpu().numpy()[l], rw, rtol=2e-6, atol=1e-7)
+    errs = [max_rel_err(y_all.cpu().numpy()[l], ys[l]) for l in range(L)]
     assert max(errs) <= TOL, errs
-    # the bf16 residual stream: equal to the oracle's except where the oracle's
-    # sum lies within the tolerance of a bf16 rounding boundary
-    xg = synth.bf16_bits_to_f32(x_out.cpu().numpy().view(np.uint16)).astype(np.float64)
-    diff = np.abs(xg - xs[-1])
-    assert np.mean(diff > 0) < 0.01 and np.all(diff <= np.abs(xs[-1]) * 2**-6 + 1e-6)
-    # spot-check the device-packed bytes of some used experts
-    used = idx_all.cpu().numpy()
-    for l in (0, L // 2, L - 1):
-        e = int(used[l, 0, 0])
-        np.testing.assert_array_equal(store.expert_bytes_at(l, e), caches[l].experts[e])
+
+
+def test_stack_wait_timeout_is_reported_and_recoverable(eo, verify_model):
+    """A grid barrier told to wait for a CTA that does not exist runs out after
+    the deadline: the status word says HFQ_ERR_TIMEOUT, the kernel winds down
+    without faulting, and the next call on the same workspace is correct."""
+    w, store = verify_model
+    H, I, E, k, L, T = w.hidden, w.inter, w.experts, w.top_k, 3, 1
+    logits = np.stack([W.logits(w, l, 7, T) for l in range(L)])
+    x0, _ = W.activations(w, 7, T)
+    d_logits = torch.from_numpy(logits).cuda()
+    d_x0 = torch.from_numpy(x0.view(np.int16)).cuda()
+    x_out = torch.empty((T, H), dtype=torch.int16, device="cuda")
+    wsb = ws(eo.hfq4_stack_workspace_bytes(T, k, H, I, E))
+    eo.hfq_set_option(eo.OPT_WAIT_TIMEOUT_NS, 20_000_000)        # 20 ms
+    try:
+        eo.hfq_set_option(eo.OPT_TEST_MISSING_ARRIVALS, 1)
+        eo.hfq4_moe_decode_stack(store.layers, d_logits, k, d_x0, T, x_out, wsb)
+        torch.cuda.synchronize()                                   # returns: nothing hung
+        with pytest.raises(eo.HfqError) as e:
+            eo.hfq_workspace_status(wsb)
+        assert e.value.status == -6
+        eo.hfq_workspace_status(wsb)                               # cleared by the read
+    finally:
+        eo.hfq_set_option(eo.OPT_WAIT_TIMEOUT_NS, 1_000_000_000)
+    x_out2, y_all, _, _, _ = _run_stack(eo, store, logits, x0, k, T, H, E, L, I)
+    caches = [moe.ExpertCache(OraclePackedLayer(w, l), H, I) for l in range(L)]
+    ys, _ = moe.residual_stack(caches, logits, synth.bf16_bits_to_f32(x0).astype(np.float64), k,
+                               route.route)
+    assert max(max_rel_err(y_all.cpu().numpy()[l], ys[l]) for l in range(L)) <= TOL
+
+
+def test_stack_launch_count(eo):
+    assert eo.hfq4_stack_launches(40, 1, 8, 2048, 512) == 1
+    assert eo.hfq4_stack_launches(40, 8, 8, 2048, 512) == 1
+    assert eo.hfq4_stack_launches(4, 1, 8, 4096, 512) == 12      # per-layer path
