@@ -57,6 +57,8 @@ _SIGS = {
     "hfq4_moe_workspace_bytes": (_sz, [_i, _i, _i, _i, _i]),
     "hfq4_moe_forward": (_i, [ctypes.POINTER(hfq4_layer), _vp, _i, _i, _vp, _vp, _i, _vp, _vp,
                               _vp, _vp, _vp, _i, _vp, _sz, _vp]),
+    "hfq4_moe_forward_noalloc": (_i, [ctypes.POINTER(hfq4_layer), _vp, _i, _i, _vp, _vp, _i,
+                                      _vp, _vp, _vp]),
     "hfq4_stack_workspace_bytes": (_sz, [_i, _i, _i, _i, _i]),
     "hfq4_stack_launches": (_i, [_i, _i, _i, _i, _i]),
     "hfq4_moe_decode_stack": (_i, [ctypes.POINTER(hfq4_layer), _i, _vp, _i, _vp, _i, _vp, _vp,
@@ -194,6 +196,15 @@ def hfq4_moe_forward(layer: Layer, x, x_dtype: int, T: int, idx, wts, k: int, y,
                                   _ptr(wts), k, _ptr(cnt), _ptr(off), _ptr(perm), _ptr(y),
                                   _ptr(y_bf16), path, _ptr(workspace), _nbytes(workspace),
                                   _stream(stream)))
+
+
+def hfq4_moe_forward_noalloc(layer: Layer, x, x_dtype: int, T: int, idx, wts, k: int, y,
+                             y_bf16=None, stream=None) -> None:
+    """hfq4_moe_forward without a workspace: for callers that cannot allocate
+    device memory (scratch is a fixed array inside the library)."""
+    _check(lib().hfq4_moe_forward_noalloc(ctypes.byref(layer.struct), _ptr(x), x_dtype, T,
+                                          _ptr(idx), _ptr(wts), k, _ptr(y), _ptr(y_bf16),
+                                          _stream(stream)))
 
 
 def hfq4_stack_workspace_bytes(T: int, k: int, hidden: int, inter: int, n_experts: int) -> int:

@@ -1,0 +1,96 @@
+// noalloc.cu - hfq4_moe_forward_noalloc: the single-layer routed-expert
+// forward for callers that must not allocate device memory.
+//
+// Some callers cannot hand this library a workspace: code running while a
+// framework captures a stream into a CUDA graph with its own allocator,
+// serving loops that forbid any allocation after start-up, plugins whose host
+// application gives them no allocator.  For them this entry point keeps its
+// scratch (the persistent kernel's control words and the h buffer) in one
+// file-scope device array, so a call allocates nothing.  The pages have no
+// counterpart to this entry point.
+#include <cstring>
+#include <mutex>
+
+#include "device.cuh"
+
+namespace hfq {
+namespace {
+
+// Largest scratch the entry point supports: the control block plus h for
+// T <= 8 tokens, k <= 16 experts per token and I <= 1024 (8*16*1024 floats).
+constexpr size_t kNoAllocHBytes = (size_t)8 * 16 * 1024 * sizeof(float);
+constexpr size_t kNoAllocCtlBytes = 36864;            // >= stack_ctl_bytes(), checked at run time
+constexpr size_t kNoAllocBytes = kNoAllocCtlBytes + kNoAllocHBytes;
+
+// Every device that loads this library holds this array until the process exits.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocBytes];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_mu;
+void *g_scratch_ptr[kMaxDevices];
+
+// Device address of the array on the current device, resolved once per
+// device (cudaGetSymbolAddress; the host-side name is only a stand-in).
+hfq_status scratch_address(void **out)
+{
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return fail(HFQ_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
+    if (dev < 0 || dev >= kMaxDevices) return fail(HFQ_ERR_UNSUPPORTED, "device %d >= %d", dev, kMaxDevices);
+    std::lock_guard<std::mutex> g(g_mu);
+    if (!g_scratch_ptr[dev]) {
+        void *p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+        if (e != cudaSuccess || !p)
+            return fail(HFQ_ERR_CUDA, "cudaGetSymbolAddress of the scratch array: %s",
+                        cudaGetErrorString(e));
+        g_scratch_ptr[dev] = p;
+    }
+    *out = g_scratch_ptr[dev];
+    return HFQ_OK;
+}
+
+}  // namespace
+}  // namespace hfq
+
+using namespace hfq;
+
+extern "C" hfq_status hfq4_moe_forward_noalloc(const hfq4_layer *layer, const void *x,
+                                               hfq_dtype x_dtype, int T, const int32_t *idx,
+                                               const float *wts, int k, float *y, void *y_bf16,
+                                               void *stream)
+{
+    if (!layer || !layer->expert_ptr) return fail(HFQ_ERR_ARG, "layer or expert_ptr is null");
+    hfq_status st = check_shape(layer->hidden, layer->inter, layer->n_experts, k);
+    if (st) return st;
+    if (!x || !idx || !wts || !y) return fail(HFQ_ERR_ARG, "hfq4_moe_forward_noalloc: null pointer");
+    if (x_dtype != HFQ_F32 && x_dtype != HFQ_BF16) return fail(HFQ_ERR_ARG, "bad x_dtype");
+    if (!aligned16(x) || !aligned16(y) || (y_bf16 && !aligned16(y_bf16)))
+        return fail(HFQ_ERR_ALIGN, "x, y and y_bf16 must be 16-byte aligned");
+    const size_t ip = (size_t)(layer->inter + HFQ4_BLOCK - 1) / HFQ4_BLOCK * HFQ4_BLOCK;
+    const size_t need_h = (size_t)T * k * ip * sizeof(float);
+    if (T < 1 || T > 8 || k > 16 || layer->inter > 1024 || need_h > kNoAllocHBytes ||
+        stack_ctl_bytes() > kNoAllocCtlBytes)
+        return fail(HFQ_ERR_UNSUPPORTED,
+                    "hfq4_moe_forward_noalloc takes T <= 8, k <= 16, inter <= 1024 (its fixed "
+                    "scratch is %zu bytes); got T=%d k=%d inter=%d", kNoAllocBytes, T, k,
+                    layer->inter);
+    int sms = 0, dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (!stack_supported(T, layer->hidden, layer->inter, k, sms))
+        return fail(HFQ_ERR_UNSUPPORTED, "shape not supported by the persistent kernel");
+    void *scratch = nullptr;
+    if ((st = scratch_address(&scratch))) return st;
+    cudaStream_t s = (cudaStream_t)stream;
+    // every call shares the array and finds the last call's contents in it:
+    // the control words must start at zero (h is fully rewritten before use)
+    cudaError_t e = cudaMemsetAsync(scratch, 0, stack_ctl_bytes(), s);
+    if (e != cudaSuccess) return fail(HFQ_ERR_CUDA, "clearing the scratch: %s", cudaGetErrorString(e));
+    float *h = reinterpret_cast<float *>(static_cast<char *>(scratch) + kNoAllocCtlBytes);
+    st = launch_stack(layer, 1, nullptr, idx, wts, x, x_dtype == HFQ_F32, T, k, nullptr, nullptr, h,
+                      y, static_cast<uint16_t *>(y_bf16), nullptr, nullptr,
+                      static_cast<unsigned *>(scratch), option_wait_timeout_ns(),
+                      option_take_extra_arrivals(), s);
+    return st ? st : ok();
+}

@@ -205,6 +205,29 @@ hfq_status hfq4_moe_decode_stack(const hfq4_layer *layers, int n_layers, const f
                                  size_t ws_bytes, void *stream);
 
 /*
+ * Allocation-free variant of hfq4_moe_forward.  The pages have no counterpart:
+ * this entry point exists for callers that cannot allocate device memory or
+ * hand the library a workspace - for example code that runs while a framework
+ * is capturing a stream into a CUDA graph with its own allocator, serving
+ * loops that forbid any allocation after start-up, or plugins whose host
+ * application gives them no allocator.  It computes the same y as
+ * hfq4_moe_forward (same kernel, same arguments minus the workspace and path)
+ * and allocates nothing: its scratch is one fixed array of device memory
+ * inside the library (548 KiB; every GPU that loads the library holds it until
+ * the process exits).
+ *   Limits: 1 <= T <= 8, k <= 16, inter <= 1024, hidden <= 2048; anything
+ *   larger returns HFQ_ERR_UNSUPPORTED naming the limit.
+ *   The first call on a device looks up the array's device address for that
+ *   device (with that device current); make that first call before any stream
+ *   capture.  Each call clears the array's control words on `stream` before
+ *   launching.  All calls share the one array, so calls that overlap on the
+ *   GPU (different streams without ordering) race; order them on one stream.
+ */
+hfq_status hfq4_moe_forward_noalloc(const hfq4_layer *layer, const void *x, hfq_dtype x_dtype,
+                                    int T, const int32_t *idx, const float *wts, int k, float *y,
+                                    void *y_bf16, void *stream);
+
+/*
  * Library options (process-wide, host side):
  *   HFQ_OPT_WAIT_TIMEOUT_NS: deadline of every bounded device-side wait
  *     (grid barriers, expert counters, ring barriers), default 1 s.  When a
