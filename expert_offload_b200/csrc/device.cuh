@@ -47,6 +47,14 @@ struct WsHeader {
 };
 constexpr size_t kWsHeader = sizeof(WsHeader);   // 256 bytes
 
+// Control block at the head of a persistent kernel's workspace, in 32-bit
+// words: [0] status (the WsHeader word), [1] CTAs finished, [64 + l] grid
+// barrier after layer l, [128 + 128 l] CTAs whose h rows of layer l are
+// written.  Zero between launches: the last CTA of a launch clears what it used.
+constexpr int kCtlDone = 1, kCtlBar = 64, kCtlH = 128, kCtlHStride = 128;
+constexpr size_t kCtlWords = kCtlH + (size_t)HFQ_MAX_STACK_LAYERS * kCtlHStride;
+constexpr size_t kCtlBytes = (kCtlWords * 4 + 255) / 256 * 256;
+
 inline cudaError_t launch_check() { return cudaGetLastError(); }
 
 // Persistent decode kernel (stack.cu).
@@ -57,6 +65,24 @@ hfq_status launch_stack(const hfq4_layer *layers, int L, const float *logits, co
                         uint16_t *x_out, uint16_t *xbuf, float *h, float *y, uint16_t *y_bf16,
                         int32_t *idx_all, float *wts_all, unsigned *ctl, long long timeout_ns,
                         int extra_arrivals, cudaStream_t s);
+
+// Persistent decode kernel for one token (decode1.cu); launch_stack hands T = 1
+// to it when decode1_launch accepts the shape (else HFQ_ERR_UNSUPPORTED with no
+// launch, and the general kernel runs).
+hfq_status decode1_launch(const hfq4_layer *layers, int L, const float *logits, const int32_t *idx_in,
+                          const float *wts_in, const void *x0, bool x0_f32, int k, uint16_t *x_out,
+                          uint16_t *xbuf, float *h, float *y, uint16_t *y_bf16, int32_t *idx_all,
+                          float *wts_all, unsigned *ctl, long long timeout_ns, int extra_arrivals,
+                          cudaStream_t s);
+int sm_count();
+
+// Tensor-core expert path (tc.cu).
+size_t tc_workspace_bytes(int T, int k, int H, int I, int E);
+bool tc_supported(int H, int I);
+hfq_status launch_tc(const hfq4_layer &L, const void *x, bool x_f32, int T, int k, const int32_t *cnt,
+                     const int32_t *off, const int32_t *perm, const float *wts, float *y,
+                     uint16_t *y_bf16, void *ws, unsigned *status, long long timeout_ns,
+                     cudaStream_t s);
 
 // Library options (hfq_set_option).
 long long option_wait_timeout_ns();

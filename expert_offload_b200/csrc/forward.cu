@@ -257,7 +257,9 @@ hfq_status hfq_set_option(int option, long long value)
 size_t hfq4_moe_workspace_bytes(int T, int k, int hidden, int inter, int n_experts)
 {
     if (T < 1 || k < 1 || hidden < 1 || inter < 1 || n_experts < 1) return 0;
-    return stack_ctl_bytes() + h_bytes(T, k, inter);
+    size_t b = stack_ctl_bytes() + h_bytes(T, k, inter);
+    if (T > 8) b += tc_workspace_bytes(T, k, hidden, inter, n_experts);   // tensor-core path
+    return b;
 }
 
 hfq_status hfq4_moe_forward(const hfq4_layer *layer, const void *x, hfq_dtype x_dtype, int T,
@@ -265,27 +267,40 @@ hfq_status hfq4_moe_forward(const hfq4_layer *layer, const void *x, hfq_dtype x_
                             const int32_t *off, const int32_t *perm, float *y, void *y_bf16,
                             int path, void *workspace, size_t ws_bytes, void *stream)
 {
-    (void)cnt; (void)off; (void)perm;
     hfq_status st = check_layer(layer, k);
     if (st) return st;
     if (!x || !idx || !wts || !y) return fail(HFQ_ERR_ARG, "hfq4_moe_forward: null pointer");
     if (T < 1 || T > 65536) return fail(HFQ_ERR_UNSUPPORTED, "T=%d not in [1, 65536]", T);
     if (x_dtype != HFQ_F32 && x_dtype != HFQ_BF16) return fail(HFQ_ERR_ARG, "bad x_dtype");
-    if (path != HFQ_PATH_AUTO && path != HFQ_PATH_GEMV)
-        return fail(HFQ_ERR_UNSUPPORTED, "path %d is not available in this build", path);
+    if (path != HFQ_PATH_AUTO && path != HFQ_PATH_GEMV && path != HFQ_PATH_TC)
+        return fail(HFQ_ERR_ARG, "unknown path %d", path);
     if (!aligned16(x) || !aligned16(y) || (y_bf16 && !aligned16(y_bf16)))
         return fail(HFQ_ERR_ALIGN, "x, y and y_bf16 must be 16-byte aligned");
+    const bool grouped = cnt && off && perm;
+    if ((cnt || off || perm) && !grouped) return fail(HFQ_ERR_ARG, "cnt, off and perm go together");
     size_t need = hfq4_moe_workspace_bytes(T, k, layer->hidden, layer->inter, layer->n_experts);
+    if (path == HFQ_PATH_TC && T <= 8)
+        need += tc_workspace_bytes(T, k, layer->hidden, layer->inter, layer->n_experts);
     if ((st = check_ws(workspace, ws_bytes, need))) return st;
-    float *h = reinterpret_cast<float *>(static_cast<char *>(workspace) + stack_ctl_bytes());
-    if (stack_supported(T, layer->hidden, layer->inter, k, num_sms_fwd())) {
+    char *wsb = static_cast<char *>(workspace);
+    float *h = reinterpret_cast<float *>(wsb + stack_ctl_bytes());
+    cudaStream_t s = (cudaStream_t)stream;
+    const bool use_tc = path == HFQ_PATH_TC || (path == HFQ_PATH_AUTO && T > 8 && grouped);
+    if (use_tc) {
+        if (!grouped)
+            return fail(HFQ_ERR_ARG, "the tensor-core path needs cnt, off and perm from moe_route");
+        if (!tc_supported(layer->hidden, layer->inter))
+            return fail(HFQ_ERR_UNSUPPORTED, "tensor-core path: hidden and inter must be multiples of 128");
+        st = launch_tc(*layer, x, x_dtype == HFQ_F32, T, k, cnt, off, perm, wts, y,
+                       static_cast<uint16_t *>(y_bf16), wsb + stack_ctl_bytes() + h_bytes(T, k, layer->inter),
+                       static_cast<unsigned *>(workspace), option_wait_timeout_ns(), s);
+    } else if (stack_supported(T, layer->hidden, layer->inter, k, num_sms_fwd())) {
         st = launch_stack(layer, 1, nullptr, idx, wts, x, x_dtype == HFQ_F32, T, k, nullptr,
                           nullptr, h, y, static_cast<uint16_t *>(y_bf16), nullptr, nullptr,
                           static_cast<unsigned *>(workspace), option_wait_timeout_ns(),
-                          option_take_extra_arrivals(), (cudaStream_t)stream);
+                          option_take_extra_arrivals(), s);
     } else {
-        st = launch_layer(*layer, x, x_dtype, T, idx, wts, k, y, y_bf16, h, nullptr, nullptr,
-                          (cudaStream_t)stream);
+        st = launch_layer(*layer, x, x_dtype, T, idx, wts, k, y, y_bf16, h, nullptr, nullptr, s);
     }
     return st ? st : ok();
 }

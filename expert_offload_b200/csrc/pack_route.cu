@@ -209,7 +209,7 @@ __global__ void group_scatter_kernel(const int32_t *__restrict__ idx, int P, int
 {
     __shared__ int wcnt[kGroupChunk / 32][HFQ_MAX_EXPERTS];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    for (int i = tid; i < (kGroupChunk / 32) * E; i += blockDim.x) (&wcnt[0][0])[i] = 0;
+    for (int i = tid; i < (kGroupChunk / 32) * E; i += blockDim.x) wcnt[i / E][i % E] = 0;
     __syncthreads();
     const int p = blockIdx.x * kGroupChunk + tid;
     const int e = p < P ? idx[p] : -1;

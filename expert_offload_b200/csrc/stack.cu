@@ -24,7 +24,10 @@
 #include <cfloat>
 
 #include "device.cuh"
+#include "gemv.cuh"
 #include "ptx.cuh"
+#include "sync.cuh"
+#include "topk.cuh"
 
 namespace hfq {
 namespace {
@@ -39,9 +42,7 @@ constexpr int kMaxRowsW = 4;            // down rows owned by one consumer warp
 constexpr int kMaxHChunks = 2;          // 16-element h chunks per lane (I <= 1024)
 constexpr int kHsPairs = 16;            // (token, expert) h vectors staged per batch
 constexpr int kStamps = 32;             // timeline stamps per layer
-constexpr int kCtlDone = 1, kCtlBar = 64, kCtlH = 128;
-constexpr size_t kCtlWords = kCtlH + (size_t)HFQ_MAX_STACK_LAYERS * kMaxU;
-constexpr size_t kCtlBytes = (kCtlWords * 4 + 255) / 256 * 256;
+constexpr int kMaxCopies = 512;         // bulk copies per layer and CTA
 constexpr int kSmemOptin = 232448;      // 227 KB per CTA on sm_100 (static + dynamic)
 constexpr int kSmemLimit = kSmemOptin - 4096;   // dynamic budget, leaving room for static
 
@@ -85,6 +86,8 @@ struct Shared {
     int pair_row[kMaxU * kMaxT];            // h row (t*k + j) of each pair slot
     const uint8_t *ubase[kMaxU];            // base address of each selected expert
     unsigned char uloc[kMaxU];              // 1 = host-mapped
+    int4 copies[kMaxCopies];                // {src offset, bytes, dst offset, stage << 8 | u}
+    int ncopies;
     int Ul[HFQ_MAX_STACK_LAYERS];
 };
 
@@ -192,111 +195,54 @@ __device__ bool next_item(Gen &g, const Geo &geo, Item &it)
 }
 
 // ---------------------------------------------------------------- waiting
-__device__ __forceinline__ bool deadline_passed(uint64_t t0, long long timeout_ns)
+__device__ __forceinline__ WaitCtx wctx(const StackArgs &a, Shared &sh)
 {
-    return (long long)(globaltimer_ns() - t0) > timeout_ns;
+    return WaitCtx{a.ctl, a.timeout_ns, &sh.abort};
 }
 
-__device__ __forceinline__ void raise_timeout(const StackArgs &a, Shared &sh)
+__device__ __forceinline__ bool wait_counter(const StackArgs &a, Shared &sh, const unsigned *p, unsigned target)
 {
-    sh.abort = 1;
-    atomicCAS(a.ctl, 0u, (unsigned)HFQ_ERR_TIMEOUT);
+    return wait_counter_ge(wctx(a, sh), p, target);
 }
 
-// Waits until *p >= target (acquire).  False on timeout or abort.  The
-// deadline clock is read only once a wait has not completed after 64 polls.
-__device__ bool wait_counter(const StackArgs &a, Shared &sh, const unsigned *p, unsigned target)
+__device__ __forceinline__ bool wait_mbar(const StackArgs &a, Shared &sh, uint64_t *bar, uint32_t parity)
 {
-    uint64_t t0 = 0;
-    for (int it = 0;; ++it) {
-        if (ld_acquire_gpu(p) >= target) return true;
-        if (sh.abort) return false;
-        if (it == 64) t0 = globaltimer_ns();
-        if (it > 64 && (it & 63) == 0) {
-            if (*(volatile unsigned *)a.ctl != 0u) { sh.abort = 1; return false; }
-            if (deadline_passed(t0, a.timeout_ns)) { raise_timeout(a, sh); return false; }
-        }
-        if (it > 16) __nanosleep(32);
-    }
-}
-
-__device__ bool wait_mbar(const StackArgs &a, Shared &sh, uint64_t *bar, uint32_t parity)
-{
-    uint64_t t0 = 0;
-    for (int it = 0;; ++it) {
-        if (mbar_try_wait(bar, parity)) return true;
-        if (sh.abort) return false;
-        if (it == 64) t0 = globaltimer_ns();
-        if (it > 64 && (it & 15) == 0 && deadline_passed(t0, a.timeout_ns)) {
-            raise_timeout(a, sh);
-            return false;
-        }
-    }
+    return wait_mbar_phase(wctx(a, sh), bar, parity);
 }
 
 // ---------------------------------------------------------------- routing
-__device__ __forceinline__ uint32_t order_key(float f)
-{
-    uint32_t u = __float_as_uint(f + 0.0f);     // -0 -> +0
-    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
-}
-
-__device__ __forceinline__ float key_value(uint32_t k)
-{
-    return __uint_as_float((k & 0x80000000u) ? (k & 0x7fffffffu) : ~k);
-}
-
-// Top-k of one token by one warp: each lane holds M consecutive experts; k
-// rounds of a warp max over the lanes' best (ties: lower lane = lower index).
+// Top-k of one token by one warp; lanes j < k also fetch the base address of
+// the j-th selected expert when `ubase` is given.
 template <int M>
-__device__ void warp_topk(const float *__restrict__ row, int E, int k, int *sel, float *wsel)
+__device__ void warp_topk(const float *__restrict__ row, int E, int k, int *sel, float *wsel,
+                          const void *const *eptr, const uint8_t *eloc, const uint8_t **ubase,
+                          unsigned char *uloc)
 {
     const int lane = threadIdx.x & 31;
-    uint32_t key[M];
-#pragma unroll
-    for (int i = 0; i < M; ++i) {
-        int e = lane * M + i;
-        key[i] = e < E ? order_key(__ldg(row + e)) : 0u;     // 0 is below every real key
-    }
-    uint32_t taken = 0, bk = key[0];
-    int bi = 0;
-#pragma unroll
-    for (int i = 1; i < M; ++i)
-        if (key[i] > bk) { bk = key[i]; bi = i; }
-    float v0 = 0.0f, s = 0.0f, my_ex = 0.0f;
-    int my_e = 0;
-    for (int j = 0; j < k; ++j) {
-        const uint32_t m = __reduce_max_sync(0xffffffffu, bk);
-        const unsigned ball = __ballot_sync(0xffffffffu, bk == m);
-        const int win = __ffs(ball) - 1;
-        const int e = __shfl_sync(0xffffffffu, lane * M + bi, win);
-        const float v = key_value(m);
-        if (j == 0) v0 = v;
-        const float ex = __expf(v - v0);
-        s += ex;
-        if (lane == j) { my_ex = ex; my_e = e; }
-        if (lane == win) {
-            taken |= 1u << bi;
-            bool any = false;
-            bk = 0u; bi = 0;
-#pragma unroll
-            for (int i = 0; i < M; ++i)
-                if (!(taken >> i & 1u) && (!any || key[i] > bk)) { bk = key[i]; bi = i; any = true; }
-        }
-    }
+    int my_e;
+    float my_w;
+    warp_topk_lane<M>(row, E, k, my_e, my_w);
     if (lane < k) {
+        if (ubase) {
+            ubase[lane] = static_cast<const uint8_t *>(eptr[my_e]);
+            uloc[lane] = eloc ? eloc[my_e] : 0;
+        }
         sel[lane] = my_e;
-        wsel[lane] = my_ex / s;
+        wsel[lane] = my_w;
     }
 }
 
-__device__ void route_token(const float *row, int E, int k, int *sel, float *wsel)
+// ubase/uloc (nullable): for a single token, slot j's expert base address and
+// location are fetched here, in slot order.
+__device__ void route_token(const float *row, int E, int k, int *sel, float *wsel,
+                            const void *const *eptr = nullptr, const uint8_t *eloc = nullptr,
+                            const uint8_t **ubase = nullptr, unsigned char *uloc = nullptr)
 {
-    if (E <= 32) warp_topk<1>(row, E, k, sel, wsel);
-    else if (E <= 64) warp_topk<2>(row, E, k, sel, wsel);
-    else if (E <= 128) warp_topk<4>(row, E, k, sel, wsel);
-    else if (E <= 256) warp_topk<8>(row, E, k, sel, wsel);
-    else warp_topk<16>(row, E, k, sel, wsel);
+    if (E <= 32) warp_topk<1>(row, E, k, sel, wsel, eptr, eloc, ubase, uloc);
+    else if (E <= 64) warp_topk<2>(row, E, k, sel, wsel, eptr, eloc, ubase, uloc);
+    else if (E <= 128) warp_topk<4>(row, E, k, sel, wsel, eptr, eloc, ubase, uloc);
+    else if (E <= 256) warp_topk<8>(row, E, k, sel, wsel, eptr, eloc, ubase, uloc);
+    else warp_topk<16>(row, E, k, sel, wsel, eptr, eloc, ubase, uloc);
 }
 
 // Unique experts of the layer, ascending; per (u, t) the slot j (or -1).
@@ -353,7 +299,8 @@ __device__ void build_table_t1(Shared &sh, int k)
 
 // Pair slots (expert-major, tokens ascending), their h rows, and every
 // selected expert's base address and location, fetched in one round of loads.
-__device__ void finish_table(Shared &sh, int k, const void *const *eptr, const uint8_t *eloc)
+__device__ void finish_table(Shared &sh, int k, const void *const *eptr, const uint8_t *eloc,
+                             bool have_bases)
 {
     const int lane = threadIdx.x & 31, U = sh.U;
     if (lane == 0) {
@@ -369,80 +316,13 @@ __device__ void finish_table(Shared &sh, int k, const void *const *eptr, const u
         }
         sh.upair0[U] = n;
     }
-    for (int u = lane; u < U; u += 32) {
+    for (int u = lane; !have_bases && u < U; u += 32) {
         const int e = sh.uexp[u];
         sh.ubase[u] = static_cast<const uint8_t *>(eptr[e]);
         sh.uloc[u] = eloc ? eloc[e] : 0;
     }
     __syncwarp();
 }
-
-// ------------------------------------------------------------------ math
-// 32 bytes of one block's payload (64 nibbles, elements 8i..8i+7 in word i)
-// against 64 activations.  Nibble -> float: `prmt` puts the byte 0x80|q into
-// bits 16..23 of 0x3F800000, giving exactly 1 + q/128 (even elements from
-// w & 0x0F0F0F0F, odd ones from (w >> 4) & 0x0F0F0F0F); the offset 1 is
-// removed afterwards with the lane's sums of x, and the factor 128 restored.
-__device__ __forceinline__ float2 nib64_fma(const uint32_t (&w)[8], const float2 *xp)
-{
-    float2 acc[4];
-#pragma unroll
-    for (int j = 0; j < 4; ++j) acc[j] = make_float2(0.f, 0.f);
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-        const uint32_t lo = (w[i] & 0x0F0F0F0Fu) | 0x80808080u;
-        const uint32_t hi = ((w[i] >> 4) & 0x0F0F0F0Fu) | 0x80808080u;
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            float2 f;
-            f.x = __uint_as_float(__byte_perm(lo, 0x3F800000u, 0x7044u | (j << 8)));
-            f.y = __uint_as_float(__byte_perm(hi, 0x3F800000u, 0x7044u | (j << 8)));
-            acc[j] = __ffma2_rn(f, xp[4 * i + j], acc[j]);
-        }
-    }
-    return make_float2((acc[0].x + acc[1].x) + (acc[2].x + acc[3].x),
-                       (acc[0].y + acc[1].y) + (acc[2].y + acc[3].y));
-}
-
-__device__ __forceinline__ float finish_dot(float2 acc, float2 sx, float scale, float zero)
-{
-    const float sq = 128.0f * ((acc.x - sx.x) + (acc.y - sx.y));
-    return fmaf(scale, sq, zero * (sx.x + sx.y));
-}
-
-__device__ __forceinline__ void lds_words(const uint8_t *p, uint32_t (&w)[8])
-{
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        uint2 v = *reinterpret_cast<const uint2 *>(p + 8 * i);
-        w[2 * i] = v.x;
-        w[2 * i + 1] = v.y;
-    }
-}
-
-// 16 nibbles (one 8-byte chunk) against 16 values held as 8 float2.
-__device__ __forceinline__ float2 nib16_fma(uint2 v, const float2 *hp, float2 acc)
-{
-    const uint32_t wv[2] = {v.x, v.y};
-#pragma unroll
-    for (int i = 0; i < 2; ++i) {
-        const uint32_t lo = (wv[i] & 0x0F0F0F0Fu) | 0x80808080u;
-        const uint32_t hi = ((wv[i] >> 4) & 0x0F0F0F0Fu) | 0x80808080u;
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            float2 f;
-            f.x = __uint_as_float(__byte_perm(lo, 0x3F800000u, 0x7044u | (j << 8)));
-            f.y = __uint_as_float(__byte_perm(hi, 0x3F800000u, 0x7044u | (j << 8)));
-            acc = __ffma2_rn(f, hp[4 * i + j], acc);
-        }
-    }
-    return acc;
-}
-
-// Padded column of activation c in shared memory: 2 floats after every 64, so
-// the lanes' 64-wide slices start on distinct bank pairs.  Keeps even columns
-// even (8-byte aligned float2 access).
-__device__ __forceinline__ int xpad(int c) { return c + 2 * (c >> 6); }
 
 // ----------------------------------------------------------------- kernel
 __device__ __forceinline__ void consumer_bar() { asm volatile("bar.sync 1, %0;" ::"r"(kCW * 32) : "memory"); }
@@ -499,7 +379,12 @@ __global__ void __launch_bounds__(kThr, 1) stack_kernel(const __grid_constant__ 
                     sh.wsel[t][j] = a.wts_in[t * a.k + j];
                 }
             } else {
-                route_token(a.logits + ((size_t)l * a.T + t) * a.E, a.E, a.k, sh.sel[t], sh.wsel[t]);
+                if constexpr (MAXT == 1)
+                    route_token(a.logits + ((size_t)l * a.T + t) * a.E, a.E, a.k, sh.sel[t],
+                                sh.wsel[t], a.eptr[l], a.eloc[l], sh.ubase, sh.uloc);
+                else
+                    route_token(a.logits + ((size_t)l * a.T + t) * a.E, a.E, a.k, sh.sel[t],
+                                sh.wsel[t]);
             }
         }
         if (warp < kCW) {
@@ -546,7 +431,8 @@ __global__ void __launch_bounds__(kThr, 1) stack_kernel(const __grid_constant__ 
         if (warp == 0) {
             if (MAXT == 1) build_table_t1(sh, a.k);
             else build_table(sh, a.T, a.k);
-            finish_table(sh, a.k, a.eptr[l], a.eloc[l]);
+            // one token routed here: the routing warp already fetched the bases
+            finish_table(sh, a.k, a.eptr[l], a.eloc[l], MAXT == 1 && !a.idx_in);
         }
         __syncthreads();
         stamp(a, 2, l, 2);
@@ -556,52 +442,86 @@ __global__ void __launch_bounds__(kThr, 1) stack_kernel(const __grid_constant__ 
             a.idx_all[((size_t)l * a.T + warp) * a.k + lane] = sh.sel[warp][lane];
             a.wts_all[((size_t)l * a.T + warp) * a.k + lane] = sh.wsel[warp][lane];
         }
-        unsigned *hdone = a.ctl + kCtlH + (size_t)l * kMaxU;     // CTAs whose h rows are written
+        unsigned *hdone = a.ctl + kCtlH + (size_t)l * kCtlHStride;     // CTAs whose h rows are written
         int n_stages_layer = 0;
 
         if (warp == kCW) {
             // ------------------------------------------ 2. producer warp
+            // First the layer's whole copy list (no issue yet: the consumers are
+            // idle and the generator runs undisturbed), then one tight issue loop.
             Gen g{0, 0, 0, 0, U};
             Item it;
+            int nc = 0;
+            bool more;
+            while ((more = next_item(g, geo, it)) && nc + 2 <= kMaxCopies) {
+                if (lane == 0) {
+                    sh.copies[nc] = make_int4((int)it.src0, it.len0, it.off0, (it.stage << 8) | it.u);
+                    if (it.type == 0)
+                        sh.copies[nc + 1] = make_int4((int)it.src1, it.len1, it.off1, (it.stage << 8) | it.u);
+                }
+                nc += it.type == 0 ? 2 : 1;
+            }
+            if (more && lane == 0) {              // excluded on the host (stack_supported)
+                sh.abort = 1;
+                atomicCAS(a.ctl, 0u, (unsigned)HFQ_ERR_UNSUPPORTED);
+            }
+            __syncwarp();
             int cur = -1, slot = 0;
-            while (!sh.abort && next_item(g, geo, it)) {
-                if (it.stage != cur) {
+            for (int ci = 0; ci < nc && !sh.abort; ++ci) {
+                const int4 c = sh.copies[ci];
+                const int stage = c.w >> 8, u = c.w & 0xFF;
+                if (stage != cur) {
                     if (cur >= 0 && lane == 0) mbar_arrive(&sh.full[slot]);
-                    cur = it.stage;
+                    cur = stage;
                     const int seq = stage_base + cur;
                     slot = seq % NS;
                     if (seq >= NS && !wait_mbar(a, sh, &sh.empty[slot], ((seq / NS) - 1) & 1)) break;
                     fence_proxy_async_smem();
                 }
-                const uint8_t *base = sh.ubase[it.u];
-                uint8_t *dst = ring + (size_t)slot * kStage;
-                const bool host = sh.uloc[it.u] != 0;
-                for (int c = 0; c < (it.type == 0 ? 2 : 1); ++c) {
-                    const int off = c ? it.off1 : it.off0, len = c ? it.len1 : it.len0;
-                    const uint8_t *src = base + (c ? it.src1 : it.src0);
-                    if (!host) {
-                        if (lane == 0) {
-                            mbar_expect_tx(&sh.full[slot], (uint32_t)len);
-                            bulk_g2s(dst + off, src, (uint32_t)len, &sh.full[slot]);
-                        }
-                    } else {
-                        // host-mapped expert: 16-byte loads over PCIe, four in flight per lane
-                        for (int o = lane * 16; o < len; o += 32 * 16 * 4) {
-                            uint4 v[4];
-#pragma unroll
-                            for (int r = 0; r < 4; ++r)
-                                if (o + r * 512 < len) v[r] = ld_nc_v4(src + o + r * 512);
-#pragma unroll
-                            for (int r = 0; r < 4; ++r)
-                                if (o + r * 512 < len)
-                                    *reinterpret_cast<uint4 *>(dst + off + o + r * 512) = v[r];
-                        }
-                        __syncwarp();
+                const uint8_t *src = sh.ubase[u] + (uint32_t)c.x;
+                if (((uintptr_t)src & 15u) != 0) {          // bulk copies start on 16 bytes
+                    if (lane == 0) { atomicCAS(a.ctl, 0u, (unsigned)HFQ_ERR_ARG); sh.abort = 1; }
+                    break;
+                }
+                uint8_t *dst = ring + (size_t)slot * kStage + c.z;
+                const int len = c.y;
+                if (!sh.uloc[u]) {
+                    if (lane == 0) {
+                        mbar_expect_tx(&sh.full[slot], (uint32_t)len);
+                        bulk_g2s(dst, src, (uint32_t)len, &sh.full[slot]);
                     }
+                } else {
+                    // host-mapped expert: 16-byte loads over PCIe, four in flight per lane
+                    for (int o = lane * 16; o < len; o += 32 * 16 * 4) {
+                        uint4 v[4];
+#pragma unroll
+                        for (int r = 0; r < 4; ++r)
+                            if (o + r * 512 < len) v[r] = ld_nc_v4(src + o + r * 512);
+#pragma unroll
+                        for (int r = 0; r < 4; ++r)
+                            if (o + r * 512 < len) *reinterpret_cast<uint4 *>(dst + o + r * 512) = v[r];
+                    }
+                    __syncwarp();
                 }
             }
             if (cur >= 0 && lane == 0) mbar_arrive(&sh.full[slot]);
-            n_stages_layer = cur + 1;
+            n_stages_layer = g.stage + (g.fill > 0 ? 1 : 0);
+            if (a.timeline && lane == 0 && n_stages_layer <= NS) {
+                // debug timeline: when this CTA's stages land (the producer is idle now)
+                const int who = blockIdx.x == 0 ? 0 : (blockIdx.x == (int)gridDim.x / 2 ? 1 : -1);
+                if (who >= 0) {
+                    unsigned long long *tl = a.timeline + ((size_t)who * a.L + l) * kStamps;
+                    tl[21] = globaltimer_ns();
+                    for (int st = 0; st < n_stages_layer && st < 10; ++st) {
+                        const int seq = stage_base + st;
+                        uint64_t t0 = globaltimer_ns();
+                        while (!mbar_try_wait(&sh.full[seq % NS], (seq / NS) & 1) &&
+                               !deadline_passed(t0, a.timeout_ns)) {
+                        }
+                        tl[22 + st] = globaltimer_ns();
+                    }
+                }
+            }
         } else {
             // ------------------------------------------ 3. consumer warps
             float2 sx[MAXT];                        // (sum over even, sum over odd) per token
@@ -741,46 +661,66 @@ __global__ void __launch_bounds__(kThr, 1) stack_kernel(const __grid_constant__ 
                         stamp(a, 0, l, 18);
                     }
                     const int slot0 = sh.upair0[u] - sh.upair0[batch_u0];   // first pair slot of u
-                    for (int i = 0; i < it.n; ++i) {
-                        const int r = it.r0 + i, rl = r - geo.d_lo;
-                        if (dead || rl % kCW != warp) continue;
-                        const int rs = rl / kCW;
-                        const uint8_t *row = sbase + it.off0 + it.dl0 + (size_t)i * geo.rowB_d;
-                        float part[MAXT];
+                    if (!dead) {
+                        // T = 1: this lane's h chunks and their sums, loaded once for the
+                        // item; T > 1: read per row from shared memory (registers)
+                        constexpr int kHT = MAXT == 1 ? 1 : 1;
+                        float2 hv[kHT][kMaxHChunks][8];
+                        float2 hsum[kHT][kMaxHChunks];
+                        if constexpr (MAXT == 1) {
 #pragma unroll
-                        for (int t = 0; t < MAXT; ++t) part[t] = 0.f;
-#pragma unroll
-                        for (int m = 0; m < kMaxHChunks; ++m) {
-                            const int c = lane + 32 * m;
-                            if (c >= nch || c * 16 >= a.I) continue;
-                            const uint8_t *blk = row + (c >> 4) * kBlockBytes;
-                            const float2 sz = *reinterpret_cast<const float2 *>(blk);
-                            const uint2 nv = *reinterpret_cast<const uint2 *>(blk + 8 + (c & 15) * 8);
-                            int ps = slot0;
-#pragma unroll
-                            for (int t = 0; t < MAXT; ++t) {
-                                if (!(um >> t & 1u)) continue;
+                            for (int m = 0; m < kMaxHChunks; ++m) {
+                                const int c = lane + 32 * m;
+                                hsum[0][m] = make_float2(0.f, 0.f);
+                                const bool ok = c < nch && c * 16 < a.I;
                                 const float2 *hp = reinterpret_cast<const float2 *>(
-                                    hs + (size_t)ps * geo.HsRow + c * 20);
-                                ++ps;
-                                float2 hv[8];
-                                float2 s2 = make_float2(0.f, 0.f);
+                                    hs + (size_t)slot0 * geo.HsRow + (ok ? c : 0) * 20);
 #pragma unroll
                                 for (int v = 0; v < 8; ++v) {
-                                    hv[v] = hp[v];
-                                    s2.x += hv[v].x;
-                                    s2.y += hv[v].y;
+                                    hv[0][m][v] = ok ? hp[v] : make_float2(0.f, 0.f);
+                                    hsum[0][m].x += hv[0][m][v].x;
+                                    hsum[0][m].y += hv[0][m][v].y;
                                 }
-                                float2 ac = nib16_fma(nv, hv, make_float2(0.f, 0.f));
-                                part[t] += finish_dot(ac, s2, sz.x, sz.y);
                             }
                         }
+                        // the rows of this item that this warp owns, as independent chains
 #pragma unroll
-                        for (int rr = 0; rr < kMaxRowsW; ++rr)
-                            if (rr == rs)
+                        for (int rs = 0; rs < kMaxRowsW; ++rs) {
+                            const int r = geo.d_lo + warp + rs * kCW;
+                            if (r < it.r0 || r >= it.r0 + it.n) continue;
+                            const uint8_t *row = sbase + it.off0 + it.dl0 + (size_t)(r - it.r0) * geo.rowB_d;
 #pragma unroll
-                                for (int t = 0; t < MAXT; ++t)
-                                    if (um >> t & 1u) acc[rr][t] = fmaf(sh.uw[u][t], part[t], acc[rr][t]);
+                            for (int m = 0; m < kMaxHChunks; ++m) {
+                                const int c = lane + 32 * m;
+                                if (c >= nch || c * 16 >= a.I) continue;
+                                const uint8_t *blk = row + (c >> 4) * kBlockBytes;
+                                const float2 sz = *reinterpret_cast<const float2 *>(blk);
+                                const uint2 nv = *reinterpret_cast<const uint2 *>(blk + 8 + (c & 15) * 8);
+                                if constexpr (MAXT == 1) {
+                                    const float part = finish_dot(nib16_fma(nv, hv[0][m]), hsum[0][m], sz.x, sz.y);
+                                    acc[rs][0] = fmaf(sh.uw[u][0], part, acc[rs][0]);
+                                } else {
+                                    int ps = slot0;
+#pragma unroll
+                                    for (int t = 0; t < MAXT; ++t) {
+                                        if (!((um >> t) & 1u)) continue;
+                                        const float2 *hp = reinterpret_cast<const float2 *>(
+                                            hs + (size_t)ps * geo.HsRow + c * 20);
+                                        ++ps;
+                                        float2 h8[8];
+                                        float2 s2 = make_float2(0.f, 0.f);
+#pragma unroll
+                                        for (int v = 0; v < 8; ++v) {
+                                            h8[v] = hp[v];
+                                            s2.x += h8[v].x;
+                                            s2.y += h8[v].y;
+                                        }
+                                        const float part = finish_dot(nib16_fma(nv, h8), s2, sz.x, sz.y);
+                                        acc[rs][t] = fmaf(sh.uw[u][t], part, acc[rs][t]);
+                                    }
+                                }
+                            }
+                        }
                     }
                 }
             }
@@ -853,23 +793,12 @@ __global__ void __launch_bounds__(kThr, 1) stack_kernel(const __grid_constant__ 
         if (*(volatile unsigned *)a.ctl == 0u) {
             for (int l = tid; l < a.L && l < HFQ_MAX_STACK_LAYERS; l += kThr) {
                 a.ctl[kCtlBar + l] = 0u;
-                a.ctl[kCtlH + (size_t)l * kMaxU] = 0u;
+                a.ctl[kCtlH + (size_t)l * kCtlHStride] = 0u;
             }
             __syncthreads();
             if (tid == 0) { __threadfence(); a.ctl[kCtlDone] = 0u; }
         }
     }
-}
-
-int sm_count()
-{
-    static int n = 0;
-    if (!n) {
-        int dev = 0;
-        cudaGetDevice(&dev);
-        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-    }
-    return n;
 }
 
 size_t smem_for(int T, int H, int I, int n_stages, int maxt)
@@ -884,12 +813,33 @@ size_t smem_for(int T, int H, int I, int n_stages, int maxt)
 
 }  // namespace
 
+int sm_count()
+{
+    static int n = 0;
+    if (!n) {
+        int dev = 0;
+        cudaGetDevice(&dev);
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    }
+    return n;
+}
+
 // Whether the persistent kernel handles this shape (else the per-layer path).
 bool stack_supported(int T, int H, int I, int k, int G)
 {
     if (T < 1 || T > kMaxT || T * k > kMaxU) return false;
+    if (expert_bytes(H, I) % 16) return false;                  // 16-byte aligned experts
     if (H > 2048 || I > 1024) return false;                     // lane slices in registers
     if ((H + G - 1) / G > kMaxRowsW * kCW) return false;
+    // bulk copies of one layer in one CTA: two per gate/up item, one per down item
+    {
+        const int nbH = (H + kBlock - 1) / kBlock, nbI = (I + kBlock - 1) / kBlock;
+        const int n_gu = (kStage / 2 - 16) / (nbH * kBlockBytes), n_d = (kStage - 16) / (nbI * kBlockBytes);
+        if (n_gu < 1 || n_d < 1) return false;
+        const int gu_rows = (I + G - 1) / G, d_rows = (H + G - 1) / G;
+        const int per_u = 2 * ((gu_rows + n_gu - 1) / n_gu) + (d_rows + n_d - 1) / n_d;
+        if (T * k * per_u > kMaxCopies) return false;
+    }
     int maxt = T == 1 ? 1 : 8;
     return smem_for(T, H, I, 4, maxt) <= (size_t)kSmemLimit;
 }
@@ -902,6 +852,12 @@ hfq_status launch_stack(const hfq4_layer *layers, int L, const float *logits, co
                         int32_t *idx_all, float *wts_all, unsigned *ctl, long long timeout_ns,
                         int extra_arrivals, cudaStream_t s)
 {
+    if (T == 1) {
+        const hfq_status st = decode1_launch(layers, L, logits, idx_in, wts_in, x0, x0_f32, k, x_out, xbuf,
+                                             h, y, y_bf16, idx_all, wts_all, ctl, timeout_ns,
+                                             extra_arrivals, s);
+        if (st != HFQ_ERR_UNSUPPORTED) return st;
+    }
     StackArgs a;
     memset(&a, 0, sizeof a);
     for (int l = 0; l < L; ++l) {
@@ -937,6 +893,12 @@ hfq_status launch_stack(const hfq4_layer *layers, int L, const float *logits, co
     const size_t smem2 = smem_for(T, a.H, a.I, ns, maxt);
     if (smem2 > (size_t)dyn_limit[maxt > 1])
         return fail(HFQ_ERR_UNSUPPORTED, "stack kernel needs %zu bytes of shared memory", smem2);
+    int resident = 0;
+    cudaError_t oe = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&resident, fn, kThr, smem2);
+    if (oe != cudaSuccess || resident < 1)
+        return fail(HFQ_ERR_UNSUPPORTED, "stack kernel: no CTA fits on an SM (%s, %zu bytes of "
+                    "shared memory); the persistent launch needs one per SM",
+                    cudaGetErrorString(oe), smem2);
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(sm_count());
     cfg.blockDim = dim3(kThr);

@@ -1,0 +1,367 @@
+// tc.cu - the token-batched expert path on the fifth-generation tensor cores
+// (tcgen05), for prefill chunks where an expert sees many tokens.
+//
+// Per expert e with T_e routed (token, slot) pairs (grouped by moe_route):
+//   G = X_e Wg^T, U = X_e Wu^T   (bf16 x bf16 -> f32 in tensor memory)
+//   H_e = bf16(silu(G) * U)
+//   O = H_e Wd^T                  (bf16 x bf16 -> f32)
+//   y[t] += w_tj * O[pair]        (f32 atomic adds)
+// The weights are dequantised from HFQ4 straight into shared memory as bf16,
+// RN_bf16(fmaf(scale, q, zero)), in the canonical K-major no-swizzle layout
+// the MMA reads (8-row x 16-byte core matrices).  Prior art on the pages: the
+// gfx1151 engine README's self-written matrix-core GEMM for prefill
+// ("Windows" section); the Strata report, section "three counter-intuitive
+// conclusions": prefill is compute-bound, decode bandwidth-bound.
+#include "device.cuh"
+#include "ptx.cuh"
+
+namespace hfq {
+namespace {
+
+constexpr int kM = 128;                    // weight rows per tile (MMA M)
+constexpr int kN = 128;                    // token pairs per tile (MMA N)
+constexpr int kKC = 64;                    // K per pipeline stage (4 MMAs of K = 16)
+constexpr int kTcThr = 256;                // 8 warps
+constexpr int kTileBytes = kM * kKC * 2;   // one 128 x 64 bf16 operand tile (16 KB)
+constexpr uint32_t kLbo = (kM / 8) * 128;  // bytes between 8-element K chunks (2048)
+constexpr uint32_t kSbo = 128;             // bytes between 8-row groups
+constexpr uint32_t kTmemCols = 256;
+
+struct TcArgs {
+    const void *const *eptr;       // [E] expert base addresses
+    const int32_t *cnt, *off, *perm;
+    const float *wts;              // [T*k] routing weights, flat
+    const uint16_t *xin;           // gate/up: X_perm [T*k][H]; down: H_perm [T*k][I] (bf16)
+    uint16_t *hout;                // gate/up: H_perm out
+    float *y;                      // down: y [T][H], accumulated
+    const int32_t *item_off;       // [E+1] prefix of work items of this phase
+    unsigned *status;
+    long long timeout_ns;
+    int E, H, I, k;
+};
+
+// Offset of element (row, kk) of a 128 x 64 operand tile in the canonical layout.
+__device__ __forceinline__ uint32_t tile_off(int row, int k8)
+{
+    return (uint32_t)(row >> 3) * kSbo + (uint32_t)(row & 7) * 16u + (uint32_t)k8 * kLbo;
+}
+
+// 8 nibbles -> 8 bf16 weights RN_bf16(fmaf(scale, q, zero)), elements in order.
+__device__ __forceinline__ uint4 deq8(uint32_t w, float scale, float zero)
+{
+    const uint32_t lo = w & 0x0F0F0F0Fu, hi = (w >> 4) & 0x0F0F0F0Fu;
+    float f[8];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        // 0x4B0000qq = 2^23 + q exactly; subtracting 2^23 is exact
+        const float qe = __uint_as_float(__byte_perm(lo, 0x4B000000u, 0x7440u | j)) - 8388608.0f;
+        const float qo = __uint_as_float(__byte_perm(hi, 0x4B000000u, 0x7440u | j)) - 8388608.0f;
+        f[2 * j] = fmaf(scale, qe, zero);
+        f[2 * j + 1] = fmaf(scale, qo, zero);
+    }
+    uint4 r;
+    __nv_bfloat162 b;
+    b = __floats2bfloat162_rn(f[0], f[1]); r.x = *reinterpret_cast<uint32_t *>(&b);
+    b = __floats2bfloat162_rn(f[2], f[3]); r.y = *reinterpret_cast<uint32_t *>(&b);
+    b = __floats2bfloat162_rn(f[4], f[5]); r.z = *reinterpret_cast<uint32_t *>(&b);
+    b = __floats2bfloat162_rn(f[6], f[7]); r.w = *reinterpret_cast<uint32_t *>(&b);
+    return r;
+}
+
+__device__ bool tc_wait(const TcArgs &a, uint64_t *bar, uint32_t parity, int &abort)
+{
+    uint64_t t0 = 0;
+    for (int it = 0;; ++it) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if (it == 64) t0 = globaltimer_ns();
+        if (it > 64 && (it & 15) == 0 && (long long)(globaltimer_ns() - t0) > a.timeout_ns) {
+            abort = 1;
+            atomicCAS(a.status, 0u, (unsigned)HFQ_ERR_TIMEOUT);
+            return false;
+        }
+    }
+}
+
+// One persistent CTA per SM walks the work items (expert, row tile, token tile).
+template <bool GU>
+__global__ void __launch_bounds__(kTcThr, 1) tc_kernel(const __grid_constant__ TcArgs a)
+{
+    extern __shared__ __align__(1024) uint8_t smem[];
+    constexpr int kOps = GU ? 3 : 2;                 // operand tiles per stage (A0 [A1] B)
+    __shared__ uint64_t mma_bar[2];
+    __shared__ uint32_t tmem_slot;
+    __shared__ int s_abort;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int K = GU ? a.H : a.I, R = GU ? a.I : a.H;
+    const int rtiles = R / kM, nK = K / kKC;
+    const int rowB = (K + kBlock - 1) / kBlock * kBlockBytes;
+    const size_t mg = (size_t)a.I * ((a.H + kBlock - 1) / kBlock) * kBlockBytes;
+    const uint32_t idesc = umma_idesc_bf16(kM, kN);
+
+    if (warp == 0) {
+        tmem_alloc(&tmem_slot, kTmemCols);
+        tmem_relinquish();
+    }
+    if (tid == 0) {
+        mbar_init(&mma_bar[0], 1);
+        mbar_init(&mma_bar[1], 1);
+        s_abort = 0;
+        fence_mbar_init();
+    }
+    tc_fence_before_sync();
+    __syncthreads();
+    tc_fence_after_sync();
+    const uint32_t tmem = tmem_slot;
+    int abort = 0;
+    uint32_t commits[2] = {0u, 0u};
+    uint32_t chunk = 0;                              // stages used so far (buffer = chunk & 1)
+    const int total = a.item_off[a.E];
+
+    for (int item = blockIdx.x; item < total; item += gridDim.x) {
+        int lo = 0, hi = a.E;                        // item_off[lo] <= item < item_off[lo + 1]
+        while (hi - lo > 1) {
+            const int mid = (lo + hi) >> 1;
+            if (a.item_off[mid] <= item) lo = mid; else hi = mid;
+        }
+        const int e = lo, local = item - a.item_off[e];
+        const int rt = local % rtiles, nt = local / rtiles;
+        const int p0 = a.off[e] + nt * kN, nvalid = min(kN, a.cnt[e] - nt * kN);
+        const int r0 = rt * kM;
+        const uint8_t *base = static_cast<const uint8_t *>(a.eptr[e]);
+        const uint8_t *A0 = GU ? base : base + 2 * mg;       // gate (or down)
+        const uint8_t *A1 = base + mg;                       // up
+
+        for (int kc = 0; kc < nK; ++kc, ++chunk) {
+            const int s = chunk & 1;
+            uint8_t *st = smem + (size_t)s * kOps * kTileBytes;
+            if (commits[s] && !abort) tc_wait(a, &mma_bar[s], (commits[s] - 1) & 1, abort);
+            const int blk = (kc * kKC) / kBlock, sub = ((kc * kKC) % kBlock) / 2;   // nibble byte
+            if (!abort) {
+                // weights: each thread one row (gate/up) or half a row (down)
+                const int row = GU ? (tid & (kM - 1)) : (tid & (kM - 1));
+                const int which = tid >> 7;                  // gate/up: matrix; down: K half
+                const uint8_t *A = (GU && which) ? A1 : A0;
+                const uint8_t *rp = A + (size_t)(r0 + row) * rowB + (size_t)blk * kBlockBytes;
+                const float2 sz = __ldg(reinterpret_cast<const float2 *>(rp));
+                uint8_t *dst = st + (GU && which ? kTileBytes : 0);
+                if (GU) {
+                    uint2 w[4];
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) w[i] = __ldg(reinterpret_cast<const uint2 *>(rp + 8 + sub + 8 * i));
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        *reinterpret_cast<uint4 *>(dst + tile_off(row, 2 * i)) = deq8(w[i].x, sz.x, sz.y);
+                        *reinterpret_cast<uint4 *>(dst + tile_off(row, 2 * i + 1)) = deq8(w[i].y, sz.x, sz.y);
+                    }
+                } else {
+                    uint2 w[2];
+#pragma unroll
+                    for (int i = 0; i < 2; ++i)
+                        w[i] = __ldg(reinterpret_cast<const uint2 *>(rp + 8 + sub + 16 * which + 8 * i));
+#pragma unroll
+                    for (int i = 0; i < 2; ++i) {
+                        *reinterpret_cast<uint4 *>(dst + tile_off(row, 4 * which + 2 * i)) = deq8(w[i].x, sz.x, sz.y);
+                        *reinterpret_cast<uint4 *>(dst + tile_off(row, 4 * which + 2 * i + 1)) = deq8(w[i].y, sz.x, sz.y);
+                    }
+                }
+                // activations: 128 token rows x 64 values, 16 bytes per piece
+                uint8_t *bt = st + (size_t)(kOps - 1) * kTileBytes;
+#pragma unroll
+                for (int i = 0; i < (kN * kKC / 8) / kTcThr; ++i) {
+                    const int id = tid + i * kTcThr;
+                    const int n = id & (kN - 1), k8 = id >> 7;
+                    uint4 v = make_uint4(0u, 0u, 0u, 0u);
+                    if (n < nvalid)
+                        v = __ldg(reinterpret_cast<const uint4 *>(a.xin + (size_t)(p0 + n) * K + kc * kKC + k8 * 8));
+                    *reinterpret_cast<uint4 *>(bt + tile_off(n, k8)) = v;
+                }
+            }
+            fence_proxy_async_smem();
+            __syncthreads();
+            if (tid == 0 && !abort && !s_abort) {
+                tc_fence_after_sync();
+                const uint8_t *bt = st + (size_t)(kOps - 1) * kTileBytes;
+#pragma unroll
+                for (int ks = 0; ks < kKC / 16; ++ks) {
+                    const uint64_t bd = umma_desc(bt + 2 * ks * kLbo, kLbo, kSbo);
+                    umma_bf16(tmem, umma_desc(st + 2 * ks * kLbo, kLbo, kSbo), bd, idesc,
+                              (kc | ks) != 0);
+                    if (GU)
+                        umma_bf16(tmem + kN, umma_desc(st + kTileBytes + 2 * ks * kLbo, kLbo, kSbo),
+                                  bd, idesc, (kc | ks) != 0);
+                }
+                umma_commit(&mma_bar[s]);
+            }
+            ++commits[s];
+            if (abort && tid == 0) s_abort = 1;
+        }
+        // all MMAs of the item are complete once its last commit has arrived
+        const int sl = (chunk - 1) & 1;
+        if (!abort && !s_abort) tc_wait(a, &mma_bar[sl], (commits[sl] - 1) & 1, abort);
+        tc_fence_after_sync();
+        if (!abort && !s_abort) {
+            const int lg = warp & 3, half = warp >> 2;          // TMEM lane group, column half
+            const int r = lg * 32 + lane;
+            const uint32_t trow = tmem + ((uint32_t)(lg * 32) << 16);
+#pragma unroll 1
+            for (int c = half * (kN / 2); c < (half + 1) * (kN / 2); c += 16) {
+                float g[16], u[16];
+                tmem_ld16(trow + c, g);
+                if (GU) tmem_ld16(trow + kN + c, u);
+                tmem_ld_wait();
+#pragma unroll
+                for (int j = 0; j < 16; ++j) {
+                    const int n = c + j;
+                    if (n >= nvalid) break;
+                    const int p = p0 + n;
+                    if (GU) {
+                        a.hout[(size_t)p * a.I + r0 + r] = float_to_bf16_bits(silu(g[j]) * u[j]);
+                    } else {
+                        const int pe = a.perm[p];
+                        atomicAdd(a.y + (size_t)(pe / a.k) * a.H + r0 + r, a.wts[pe] * g[j]);
+                    }
+                }
+            }
+        }
+        tc_fence_before_sync();
+        __syncthreads();
+        if (s_abort) abort = 1;
+    }
+    // no MMA may still write tensor memory when it is freed
+    if (tid == 0 && chunk) {
+        const int sl = (chunk - 1) & 1;
+        int dummy = 0;
+        tc_wait(a, &mma_bar[sl], (commits[sl] - 1) & 1, dummy);
+    }
+    tc_fence_before_sync();
+    __syncthreads();
+    tc_fence_after_sync();
+    if (warp == 0) tmem_dealloc(tmem, kTmemCols);
+}
+
+// Work items per expert: ceil(cnt/kN) token tiles x (rows/kM) row tiles, for
+// the gate/up phase (rows = I) and the down phase (rows = H); exclusive scans.
+__global__ void tc_plan_kernel(const int32_t *__restrict__ cnt, int E, int I, int H,
+                               int32_t *__restrict__ gu_off, int32_t *__restrict__ dn_off)
+{
+    __shared__ int s_gu[HFQ_MAX_EXPERTS], s_dn[HFQ_MAX_EXPERTS];
+    for (int e = threadIdx.x; e < E; e += blockDim.x) {
+        const int tiles = (cnt[e] + kN - 1) / kN;
+        s_gu[e] = tiles * (I / kM);
+        s_dn[e] = tiles * (H / kM);
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        int a = 0, b = 0;
+        for (int e = 0; e < E; ++e) {
+            gu_off[e] = a; dn_off[e] = b;
+            a += s_gu[e]; b += s_dn[e];
+        }
+        gu_off[E] = a; dn_off[E] = b;
+    }
+}
+
+// X_perm[q] = x[token of pair perm[q]] as bf16 (16 bytes per thread step).
+__global__ void tc_gather_kernel(const void *__restrict__ x, int x_f32, const int32_t *__restrict__ perm,
+                                 int P, int k, int H, uint16_t *__restrict__ xp)
+{
+    const size_t n8 = (size_t)P * H / 8;
+    for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n8;
+         i += (size_t)gridDim.x * blockDim.x) {
+        const size_t q = i / (H / 8), c = (i - q * (H / 8)) * 8;
+        const size_t src = (size_t)(perm[q] / k) * H + c;
+        uint4 v;
+        if (x_f32) {
+            const float4 a = __ldg(reinterpret_cast<const float4 *>(static_cast<const float *>(x) + src));
+            const float4 b = __ldg(reinterpret_cast<const float4 *>(static_cast<const float *>(x) + src) + 1);
+            __nv_bfloat162 t;
+            t = __floats2bfloat162_rn(a.x, a.y); v.x = *reinterpret_cast<uint32_t *>(&t);
+            t = __floats2bfloat162_rn(a.z, a.w); v.y = *reinterpret_cast<uint32_t *>(&t);
+            t = __floats2bfloat162_rn(b.x, b.y); v.z = *reinterpret_cast<uint32_t *>(&t);
+            t = __floats2bfloat162_rn(b.z, b.w); v.w = *reinterpret_cast<uint32_t *>(&t);
+        } else {
+            v = __ldg(reinterpret_cast<const uint4 *>(static_cast<const uint16_t *>(x) + src));
+        }
+        *reinterpret_cast<uint4 *>(xp + q * H + c) = v;
+    }
+}
+
+__global__ void tc_y_bf16_kernel(const float *__restrict__ y, size_t n, uint16_t *__restrict__ yb)
+{
+    for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
+         i += (size_t)gridDim.x * blockDim.x)
+        yb[i] = float_to_bf16_bits(y[i]);
+}
+
+int tc_sms()
+{
+    static int n = 0;
+    if (!n) {
+        int dev = 0;
+        cudaGetDevice(&dev);
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    }
+    return n;
+}
+
+}  // namespace
+
+size_t tc_workspace_bytes(int T, int k, int H, int I, int E)
+{
+    const size_t P = (size_t)T * k;
+    auto r256 = [](size_t b) { return (b + 255) / 256 * 256; };
+    return r256(P * H * 2) + r256(P * I * 2) + 2 * r256((size_t)(E + 1) * 4);
+}
+
+bool tc_supported(int H, int I)
+{
+    return H % kM == 0 && I % kM == 0 && H % kKC == 0 && I % kKC == 0;
+}
+
+hfq_status launch_tc(const hfq4_layer &L, const void *x, bool x_f32, int T, int k, const int32_t *cnt,
+                     const int32_t *off, const int32_t *perm, const float *wts, float *y,
+                     uint16_t *y_bf16, void *ws, unsigned *status, long long timeout_ns,
+                     cudaStream_t s)
+{
+    const int H = L.hidden, I = L.inter, E = L.n_experts;
+    const size_t P = (size_t)T * k;
+    auto r256 = [](size_t b) { return (b + 255) / 256 * 256; };
+    uint8_t *w = static_cast<uint8_t *>(ws);
+    uint16_t *xp = reinterpret_cast<uint16_t *>(w);
+    w += r256(P * H * 2);
+    uint16_t *hp = reinterpret_cast<uint16_t *>(w);
+    w += r256(P * I * 2);
+    int32_t *gu_off = reinterpret_cast<int32_t *>(w);
+    w += r256((size_t)(E + 1) * 4);
+    int32_t *dn_off = reinterpret_cast<int32_t *>(w);
+
+    static bool attr = false;
+    const int smem_gu = 2 * 3 * kTileBytes, smem_dn = 2 * 2 * kTileBytes;
+    if (!attr) {
+        cudaFuncSetAttribute(tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_gu);
+        cudaFuncSetAttribute(tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_dn);
+        attr = true;
+    }
+    tc_plan_kernel<<<1, 512, 0, s>>>(cnt, E, I, H, gu_off, dn_off);
+    const size_t n8 = P * H / 8;
+    tc_gather_kernel<<<(unsigned)std::min<size_t>((n8 + 255) / 256, (size_t)tc_sms() * 16), 256, 0, s>>>(
+        x, x_f32 ? 1 : 0, perm, (int)P, k, H, xp);
+    cudaMemsetAsync(y, 0, (size_t)T * H * sizeof(float), s);
+    TcArgs a;
+    a.eptr = L.expert_ptr; a.cnt = cnt; a.off = off; a.perm = perm; a.wts = wts;
+    a.status = status; a.timeout_ns = timeout_ns; a.E = E; a.H = H; a.I = I; a.k = k;
+    a.xin = xp; a.hout = hp; a.y = nullptr; a.item_off = gu_off;
+    tc_kernel<true><<<tc_sms(), kTcThr, smem_gu, s>>>(a);
+    a.xin = hp; a.hout = nullptr; a.y = y; a.item_off = dn_off;
+    tc_kernel<false><<<tc_sms(), kTcThr, smem_dn, s>>>(a);
+    if (y_bf16) {
+        const size_t n = (size_t)T * H;
+        tc_y_bf16_kernel<<<(unsigned)std::min<size_t>((n + 255) / 256, (size_t)tc_sms() * 16), 256, 0, s>>>(
+            y, n, y_bf16);
+    }
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return fail(HFQ_ERR_CUDA, "tensor-core path launch: %s", cudaGetErrorString(e));
+    return HFQ_OK;
+}
+
+}  // namespace hfq

@@ -165,12 +165,20 @@ typedef struct {
  * summed in slot order j with fp32 accumulation.
  *   x:      [T][H] in x_dtype (f32 or bf16).
  *   idx, wts: routing as written by moe_route ([T][k]).
- *   cnt, off, perm: grouping by expert; required for HFQ_PATH_TC and AUTO
- *           with T > 8, ignored otherwise (may be NULL).
+ *   cnt, off, perm: grouping by expert (from moe_route); required for
+ *           HFQ_PATH_TC; with AUTO and T > 8 they select the tensor-core
+ *           path, without them T > 8 runs the per-layer GEMV kernels.
+ *   path:   AUTO: T <= 8 -> persistent GEMV kernel; T > 8 with grouping ->
+ *           tensor cores.  GEMV forces CUDA cores; TC forces the tensor-core
+ *           path [WMMA]: weights dequantised to RN_bf16(fmaf(scale, q, zero)),
+ *           x rounded to bf16 (exact for bf16 input), f32 accumulation, h
+ *           rounded to bf16 before the down projection, y accumulated with f32
+ *           atomic adds (the order of the k slots is not fixed).
  *   y:      f32 [T][H] out.  y_bf16: optional bf16 [T][H] out (NULL = none).
  *   workspace: hfq4_moe_workspace_bytes(T, k, H, I, E) bytes of device
- *           scratch, 256-byte aligned, owned by the caller; calls that share
- *           a workspace must be ordered on one stream.
+ *           scratch (plus the same again for HFQ_PATH_TC with T <= 8),
+ *           256-byte aligned, zero-filled before first use, owned by the
+ *           caller; calls that share a workspace must be ordered on one stream.
  */
 size_t hfq4_moe_workspace_bytes(int T, int k, int hidden, int inter, int n_experts);
 hfq_status hfq4_moe_forward(const hfq4_layer *layer, const void *x, hfq_dtype x_dtype, int T,
@@ -241,7 +249,8 @@ hfq_status hfq4_moe_forward_noalloc(const hfq4_layer *layer, const void *x, hfq_
  *     launches then write %globaltimer stamps (ns) for two CTAs (CTA 0 and CTA
  *     gridDim/2), per layer: [0] layer start, [1] routed, [2] table built,
  *     [3 + s] ring stage s ready (s < 12), [16] gate/up done, [17] all h
- *     ready, [18] h staged, [19] down done, [20] layer end.
+ *     ready, [18] h staged, [19] down done, [20] layer end, [21] all copies
+ *     issued, [22 + s] bytes of stage s landed (s < 10, one token only).
  * Returns HFQ_ERR_ARG for an unknown option or a value out of range.
  */
 #define HFQ_OPT_WAIT_TIMEOUT_NS 1

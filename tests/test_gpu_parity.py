@@ -136,6 +136,15 @@ def test_route_prefill_zipf_8192(eo):
     _check_route(eo, W.logits(w, 0, 0, 8192), w.top_k)
 
 
+def test_route_grouping_with_few_experts_and_many_pairs(eo):
+    """E < 512 with more than one warp's worth of pairs per chunk (a grouping
+    table was once cleared only for E = 512)."""
+    import dataclasses
+    w = dataclasses.replace(W.WORKLOADS[4], experts=32)
+    _check_route(eo, W.zipf_logits(w, 0, 0, 256), 8)
+    _check_route(eo, np.random.default_rng(9).standard_normal((300, 100)).astype(np.float32), 6)
+
+
 def test_route_ties_and_degenerate_cases(eo):
     l = np.array([[1.0, 2.0, 2.0, 0.0, 2.0, -1.0, 2.0, 0.5]], dtype=np.float32)
     _check_route(eo, l, 3)                       # three of four tied values selected

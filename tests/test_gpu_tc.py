@@ -1,0 +1,119 @@
+"""GPU parity of the tensor-core (tcgen05) expert path for prefill chunks.
+
+The path computes the same layer with bf16 operands: weights RN_bf16 of their
+correctly rounded f32 values, bf16 activations, f32 accumulation, h rounded
+to bf16 before the down projection.  The oracle's bf16 model (moe.ExpertCache
+with tc=True) states exactly that; y must match it within 1e-3."""
+import dataclasses
+
+import numpy as np
+import pytest
+
+import synth
+from oracle import moe, route
+from synth import workloads as W
+from tests.gpu_util import TOL, OraclePackedLayer, device_fill, max_rel_err
+
+pytestmark = pytest.mark.gpu
+torch = pytest.importorskip("torch")
+
+
+@pytest.fixture(scope="module")
+def eo():
+    assert torch.cuda.is_available()
+    synth.build()
+    from expert_offload_b200 import build
+    build.build()
+    import expert_offload_b200
+    return expert_offload_b200
+
+
+def _route(eo, logits, k):
+    T, E = logits.shape
+    lg = torch.from_numpy(np.ascontiguousarray(logits)).cuda()
+    idx = torch.empty((T, k), dtype=torch.int32, device="cuda")
+    wts = torch.empty((T, k), dtype=torch.float32, device="cuda")
+    cnt = torch.empty(E, dtype=torch.int32, device="cuda")
+    off = torch.empty(E + 1, dtype=torch.int32, device="cuda")
+    perm = torch.empty(T * k, dtype=torch.int32, device="cuda")
+    rws = torch.zeros(max(256, eo.hfq_route_workspace_bytes(T, E, k)), dtype=torch.uint8,
+                      device="cuda")
+    eo.moe_route(lg, T, E, k, idx, wts, cnt, off, perm, rws)
+    return idx, wts, cnt, off, perm
+
+
+def _forward(eo, layer, x_bits, T, k, routed, path, H, I, E):
+    idx, wts, cnt, off, perm = routed
+    y = torch.full((T, H), float("nan"), dtype=torch.float32, device="cuda")
+    need = eo.hfq4_moe_workspace_bytes(T, k, H, I, E) * (2 if path == eo.PATH_TC and T <= 8 else 1)
+    ws = torch.zeros(need, dtype=torch.uint8, device="cuda")
+    eo.hfq4_moe_forward(layer, torch.from_numpy(x_bits.view(np.int16)).cuda(), eo.HFQ_BF16, T, idx,
+                        wts, k, y, ws, cnt=cnt, off=off, perm=perm, path=path)
+    torch.cuda.synchronize()
+    eo.hfq_workspace_status(ws)
+    return y.cpu().numpy()
+
+
+@pytest.fixture(scope="module")
+def small_layer(eo):
+    """32 experts at full H = 2048, I = 512, Zipf(1.1) routing so that the head
+    experts span several 128-token tiles."""
+    from expert_offload_b200.model import ExpertStore
+    w = dataclasses.replace(W.WORKLOADS[4], experts=32)
+    store = ExpertStore(torch, 1, 32, w.hidden, w.inter, device_fill(torch, w))
+    return w, store
+
+
+def test_tc_path_all_tokens(eo, small_layer):
+    w, store = small_layer
+    H, I, E, k, T = w.hidden, w.inter, w.experts, w.top_k, 256
+    logits = W.zipf_logits(w, 0, 0, T)
+    x, _ = W.activations(w, 0, T)
+    routed = _route(eo, logits, k)
+    cnt = routed[2].cpu().numpy()
+    assert cnt.max() > 128 and cnt.sum() == T * k          # multi-tile and ragged experts
+    y = _forward(eo, store.layers[0], x, T, k, routed, eo.PATH_TC, H, I, E)
+    ridx, rw = route.route(logits, k)
+    np.testing.assert_array_equal(routed[0].cpu().numpy(), ridx)
+    cache = moe.ExpertCache(OraclePackedLayer(w, 0), H, I, tc=True)
+    ref = moe.moe_layer(cache, H, I, synth.bf16_bits_to_f32(x).astype(np.float64), ridx, rw)
+    err = max_rel_err(y, ref)
+    assert err <= TOL, err
+
+
+def test_tc_and_gemv_paths_agree(eo, small_layer):
+    w, store = small_layer
+    H, I, E, k, T = w.hidden, w.inter, w.experts, w.top_k, 40
+    logits = W.zipf_logits(w, 0, 5000, T)
+    x, _ = W.activations(w, 5000, T)
+    routed = _route(eo, logits, k)
+    y_tc = _forward(eo, store.layers[0], x, T, k, routed, eo.PATH_TC, H, I, E)
+    y_gv = _forward(eo, store.layers[0], x, T, k, routed, eo.PATH_GEMV, H, I, E)
+    ridx, rw = route.route(logits, k)
+    xv = synth.bf16_bits_to_f32(x).astype(np.float64)
+    ref_exact = moe.moe_layer(moe.ExpertCache(OraclePackedLayer(w, 0), H, I), H, I, xv, ridx, rw)
+    assert max_rel_err(y_gv, ref_exact) <= TOL
+    # the bf16 model and the exact layer differ by the bf16 rounding of weights and h
+    assert max_rel_err(y_tc, ref_exact) <= 2e-2
+
+
+@pytest.mark.slow
+def test_tc_prefill_chunk_8192_sampled(eo):
+    """The 512-expert, 8192-token prefill chunk at full size; the oracle checks
+    a sample of tokens one by one."""
+    from expert_offload_b200.model import ExpertStore
+    w = W.WORKLOADS[4]
+    H, I, E, k, T = w.hidden, w.inter, w.experts, w.top_k, 8192
+    store = ExpertStore(torch, 1, E, H, I, device_fill(torch, w))
+    logits = W.zipf_logits(w, 0, 0, T)
+    x, _ = W.activations(w, 0, T)
+    routed = _route(eo, logits, k)
+    y = _forward(eo, store.layers[0], x, T, k, routed, eo.PATH_AUTO, H, I, E)
+    assert np.all(np.isfinite(y))
+    sample = [0, 1, 2, 4095, 8191]
+    ridx, rw = route.route(logits[sample], k)
+    np.testing.assert_array_equal(routed[0].cpu().numpy()[sample], ridx)
+    cache = moe.ExpertCache(OraclePackedLayer(w, 0), H, I, tc=True)
+    ref = moe.moe_layer(cache, H, I, synth.bf16_bits_to_f32(x[sample]).astype(np.float64), ridx, rw)
+    err = max_rel_err(y[sample], ref)
+    assert err <= TOL, err

@@ -88,3 +88,84 @@ def test_ring_items_cover_what_consumers_read(T, H, I, k, G):
                     off += ln
                 fill += need
                 r0 += n
+
+
+# ----------------------------------------------------------------------------
+# decode1.cu: the one-token persistent kernel.  Restates its shared-memory
+# layout (launcher) and per-CTA spans (kernel) and checks every bulk copy and
+# shared-memory read against them.
+D1_W, D1_MAX_DROWS, D1_SMEM = 8, 16, 232448
+D1_SHARED = 16 * 8 * 2 + 16 * 8 + 16 * 4 + 16      # D1Shared, upper bound
+
+
+def up16(b):
+    return (b + 15) // 16 * 16
+
+
+def decode1_layout(H, I, E, k, G):
+    nbH, nbI = -(-H // 256), -(-I // 256)
+    Hp = nbH * 256
+    rowB_gu, rowB_d = nbH * K_BB, nbI * K_BB
+    gspan = up16(-(-I // G) * rowB_gu + 15)
+    dspan = up16(-(-H // G) * rowB_d + 15)
+    slot = (2 * gspan + dspan + 127) // 128 * 128
+    off = k * slot
+    lay = dict(slot=slot, up=gspan, down=2 * gspan, gspan=gspan, dspan=dspan, xs=off)
+    off += up16((Hp + 2 * (Hp >> 6)) * 4)
+    lay["ptab"] = off
+    off += 2 * E * 8
+    lay["ltab_stride"] = up16(E)
+    lay["ltab"] = off
+    off += 2 * lay["ltab_stride"]
+    lay["ysh"] = off
+    off += D1_W * D1_MAX_DROWS * 4
+    lay["sh"] = up16(off)
+    lay["total"] = lay["sh"] + D1_SHARED
+    return lay
+
+
+def decode1_accepts(H, I, E, k, G):
+    return (1 <= k <= 16 and H <= 2048 and H % 8 == 0 and I <= 1024 and I % 16 == 0
+            and E <= 512 and E % 16 == 0 and -(-H // G) <= D1_MAX_DROWS)
+
+
+@pytest.mark.parametrize("H,I,E,k,G", [(2048, 512, 256, 8, 148), (2048, 512, 512, 8, 148),
+                                       (256, 128, 16, 4, 148), (2048, 768, 128, 8, 148),
+                                       (2048, 512, 256, 16, 148), (1024, 1024, 64, 6, 132)])
+def test_decode1_copies_and_reads_stay_in_their_slot(H, I, E, k, G):
+    assert decode1_accepts(H, I, E, k, G)
+    lay = decode1_layout(H, I, E, k, G)
+    assert lay["total"] <= D1_SMEM
+    for key in ("slot", "up", "down", "xs", "ptab", "ltab", "ysh", "sh"):
+        assert lay[key] % 16 == 0, key              # bulk-copy and cp.async destinations
+    nbH, nbI = -(-H // 256), -(-I // 256)
+    rowB_gu, rowB_d = nbH * K_BB, nbI * K_BB
+    mg = I * rowB_gu
+    eb = 2 * mg + H * rowB_d                # expert bytes; the kernels take multiples of 16
+    assert eb % 16 == 0
+    for c in range(G):
+        gu_lo, gu_hi = c * I // G, (c + 1) * I // G
+        d_lo, d_hi = c * H // G, (c + 1) * H // G
+        assert d_hi - d_lo <= D1_MAX_DROWS
+        for off, n, rowB, region, cap in ((gu_lo * rowB_gu, gu_hi - gu_lo, rowB_gu, "up", lay["gspan"]),
+                                          (mg + gu_lo * rowB_gu, gu_hi - gu_lo, rowB_gu, "up", lay["gspan"]),
+                                          (2 * mg + d_lo * rowB_d, d_hi - d_lo, rowB_d, "down", lay["dspan"])):
+            src, ln, delta = span16(off, n * rowB)
+            if n == 0:
+                continue
+            assert src % 16 == 0 and ln % 16 == 0 and ln <= cap
+            assert src + ln <= eb                       # never past the expert's last byte
+            assert delta % 8 == 0                       # float2 scale/zero and uint2 nibble reads
+            # reads: rows r < n, blocks of 136 bytes, within the copied span
+            last = delta + (n - 1) * rowB + rowB
+            assert last <= ln
+    # the next slot starts after the largest span set
+    assert 2 * lay["gspan"] + lay["dspan"] <= lay["slot"]
+    assert lay["xs"] + up16((nbH * 256 + 2 * (nbH * 256 >> 6)) * 4) <= lay["ptab"]
+
+
+def test_decode1_declines_shapes_outside_its_registers():
+    assert not decode1_accepts(4096, 512, 256, 8, 148)      # a lane covers 64 of at most 2048 columns
+    assert not decode1_accepts(2048, 2048, 256, 8, 148)     # two 16-value h chunks per lane
+    assert not decode1_accepts(2048, 512, 256, 17, 148)     # two slots per warp
+    assert not decode1_accepts(2048, 512, 250, 8, 148)      # 16-byte table copies
