@@ -25,6 +25,8 @@
 // The expert address table of layer l+1 comes into shared memory (cp.async)
 // while layer l runs.  Every wait is bounded (sync.cuh); on expiry the status
 // word holds HFQ_ERR_TIMEOUT and every CTA winds down.
+#include <algorithm>
+
 #include "device.cuh"
 #include "gemv.cuh"
 #include "ptx.cuh"
@@ -37,9 +39,10 @@ namespace {
 constexpr int kW = 8;                   // warps
 constexpr int kThr = kW * 32;
 constexpr int kMaxK = 16;               // routed slots, two per warp
-constexpr int kMaxDRows = 16;           // down rows per CTA
-constexpr int kMaxHChunks = 2;          // 16-value h chunks per lane (I <= 1024)
+constexpr int kMaxDRows = 16;           // down rows per CTA (one batched warp reduction)
+constexpr int kGuRows = 4;              // gate/up rows per batched warp reduction
 constexpr int kXLoads = 4;              // 16-byte input loads per thread (H <= 2048)
+constexpr int kHLoads = 8;              // 16-byte h loads per lane and slot (I <= 1024)
 constexpr int kStamps = 32;             // timeline stamps per layer
 constexpr int kSmemOptin = 232448;      // 227 KB per CTA on sm_100
 
@@ -80,6 +83,11 @@ struct D1Shared {
     int armed;                        // layers whose slot barriers were armed
 };
 
+// Padded f32 column of activation c in shared memory: 4 floats after every 64,
+// so the lanes' 64-wide slices start on distinct bank quads and stay 16-byte
+// aligned (128-bit loads).
+__device__ __forceinline__ int xp4(int c) { return c + 4 * (c >> 6); }
+
 // One contiguous byte range of an expert, widened to 16-byte boundaries.
 struct Span {
     uint32_t src;     // 16-aligned offset within the expert
@@ -102,6 +110,20 @@ __device__ __forceinline__ void stamp(const D1Args &a, int l, int s)
     if (a.timeline && threadIdx.x == 0 && l < a.L) {
         const int slot = blockIdx.x == 0 ? 0 : (blockIdx.x == gridDim.x / 2 ? 1 : -1);
         if (slot >= 0) a.timeline[((size_t)slot * a.L + l) * kStamps + s] = globaltimer_ns();
+    }
+}
+
+// Debug timeline, thread `who` of CTAs 0 and G/2: %globaltimer once `dep`
+// (a value the stamp waits for) is available.
+__device__ __forceinline__ void stamp_dep(const D1Args &a, int l, int s, bool who, float dep)
+{
+    if (a.timeline && who && l < a.L) {
+        const int slot = blockIdx.x == 0 ? 0 : (blockIdx.x == gridDim.x / 2 ? 1 : -1);
+        if (slot >= 0) {
+            uint64_t t;
+            asm volatile("{ .reg .f32 d; mov.b32 d, %1; mov.u64 %0, %%globaltimer; }" : "=l"(t) : "f"(dep));
+            a.timeline[((size_t)slot * a.L + l) * kStamps + s] = t;
+        }
     }
 }
 
@@ -154,7 +176,7 @@ __global__ void __launch_bounds__(kThr, 1) decode1_kernel(const __grid_constant_
     const Span sd = span_of(2 * mg + (size_t)d_lo * rowB_d, (size_t)n_d * rowB_d);
 
     uint8_t *slots = smem;
-    float *xs = reinterpret_cast<float *>(smem + a.xs_off);          // [xpad(Hp)] f32
+    float *xs = reinterpret_cast<float *>(smem + a.xs_off);          // [xp4(Hp)] f32
     uint8_t *ptab = smem + a.ptab_off;                                // [2][E] addresses
     uint8_t *ltab = smem + a.ltab_off;                                // [2][ltab_stride]
     float *ysh = reinterpret_cast<float *>(smem + a.ysh_off);        // [kW][kMaxDRows]
@@ -170,7 +192,7 @@ __global__ void __launch_bounds__(kThr, 1) decode1_kernel(const __grid_constant_
         sh.armed = 0;
         fence_mbar_init();
     }
-    for (int i = H + tid; i < Hp; i += kThr) xs[xpad(i)] = 0.0f;   // padding, never rewritten
+    for (int i = H + tid; i < Hp; i += kThr) xs[xp4(i)] = 0.0f;   // padding, never rewritten
     if (warp == 0) fetch_table(a, 0, ptab, ltab);
     __syncthreads();
 
@@ -181,6 +203,7 @@ __global__ void __launch_bounds__(kThr, 1) decode1_kernel(const __grid_constant_
             // ------------------------------------------ 1a. route, issue copies
             cp_async_wait_all();
             __syncwarp();
+            stamp_dep(a, l, 29, lane == 0, 0.f);
             int e = -1;
             float w = 0.0f;
             if (a.idx_in) {
@@ -188,7 +211,7 @@ __global__ void __launch_bounds__(kThr, 1) decode1_kernel(const __grid_constant_
             } else {
                 warp_route(a.logits + (size_t)l * E, E, k, e, w);
             }
-            if (l + 1 < a.L) fetch_table(a, l + 1, ptab, ltab);
+            stamp_dep(a, l, 2, lane == 0, w);
             bool bad = lane < k && (unsigned)e >= (unsigned)E;
             const uint8_t *base = nullptr;
             int loc = 0;
@@ -211,6 +234,7 @@ __global__ void __launch_bounds__(kThr, 1) decode1_kernel(const __grid_constant_
             }
             const unsigned hm = __ballot_sync(0xffffffffu, lane < k && loc != 0);
             __syncwarp();
+            stamp_dep(a, l, 25, lane == 0, 0.f);
             if (!sh.abort) {
                 // the slots were last read by the generic proxy (previous layer)
                 fence_proxy_async_smem();
@@ -225,6 +249,7 @@ __global__ void __launch_bounds__(kThr, 1) decode1_kernel(const __grid_constant_
                     }
                 }
                 __syncwarp();
+                stamp_dep(a, l, 26, lane == 0, 0.f);
                 if (lane < k && !loc) {
                     uint8_t *slot = slots + (size_t)lane * a.slot_bytes;
                     if (sg.len) bulk_g2s(slot, base + sg.src, (uint32_t)sg.len, &sh.gu_bar[lane]);
@@ -232,7 +257,13 @@ __global__ void __launch_bounds__(kThr, 1) decode1_kernel(const __grid_constant_
                     if (sd.len) bulk_g2s(slot + a.down_off, base + sd.src, (uint32_t)sd.len, &sh.d_bar[lane]);
                 }
                 if (lane == 0) { sh.armed = l + 1; sh.hostmask = hm; }
+                __syncwarp();
+                stamp_dep(a, l, 27, lane == 0, 0.f);
             }
+            // next layer's table, after the copies: the proxy fence above must
+            // not wait for it
+            if (l + 1 < a.L) fetch_table(a, l + 1, ptab, ltab);
+            stamp_dep(a, l, 3, lane == 0, 0.f);
         } else {
             // ------------------------------------------ 1b. layer input -> xs
             const void *xin = l == 0 ? a.x0 : (const void *)(a.xbuf + (size_t)(l & 1) * H);
@@ -249,7 +280,7 @@ __global__ void __launch_bounds__(kThr, 1) decode1_kernel(const __grid_constant_
             for (int q = 0; q < kXLoads; ++q) {
                 const int i = tid - 32 + q * (kThr - 32);
                 if (i >= nld) continue;
-                float2 *dst = reinterpret_cast<float2 *>(xs + xpad(i * per));
+                float2 *dst = reinterpret_cast<float2 *>(xs + xp4(i * per));
                 if (f32) {
                     dst[0] = make_float2(__uint_as_float(v[q].x), __uint_as_float(v[q].y));
                     dst[1] = make_float2(__uint_as_float(v[q].z), __uint_as_float(v[q].w));
@@ -260,23 +291,36 @@ __global__ void __launch_bounds__(kThr, 1) decode1_kernel(const __grid_constant_
                         dst[r] = make_float2(__uint_as_float(w4[r] << 16), __uint_as_float(w4[r] & 0xFFFF0000u));
                 }
             }
+            stamp_dep(a, l, 4, tid == 32, __uint_as_float(v[0].x & 0x7F7FFFFFu));
         }
         if (__syncthreads_or(sh.abort)) break;
         stamp(a, l, 1);
 
         // ---------------------------------------------- 2. gate/up rows
-        // lane: block pb of the row, quarter pq (64 weights, 32 payload bytes)
+        // lane: block pb of the row, quarter pq (64 weights, 32 payload bytes).
+        // Its 64 activations stay in registers as scaled bf16 pairs (gemv.cuh,
+        // nib8_dot_bf16); the 2 * kGuRows dots of a row group run side by side.
         const int pb = lane >> 2, pq = lane & 3;
         const bool has_piece = pb < nbH;
-        float2 xr[32];
-        float2 sx = make_float2(0.f, 0.f);
+        uint32_t X[32];
+        float sxp = 0.0f;                       // sum of the piece's activations
+        int xs_exp = 0;                         // the piece's scale exponent
         {
-            const float2 *xp = reinterpret_cast<const float2 *>(xs + xpad(has_piece ? pb * kBlock + pq * 64 : 0));
+            const float4 *xq = reinterpret_cast<const float4 *>(xs + xp4(has_piece ? pb * kBlock + pq * 64 : 0));
+            float m = 0.0f;
 #pragma unroll
-            for (int i = 0; i < 32; ++i) {
-                xr[i] = has_piece ? xp[i] : make_float2(0.f, 0.f);
-                sx.x += xr[i].x;
-                sx.y += xr[i].y;
+            for (int i = 0; i < 16; ++i) {
+                const float4 q = has_piece ? xq[i] : make_float4(0.f, 0.f, 0.f, 0.f);
+                sxp += (q.x + q.y) + (q.z + q.w);
+                m = fmaxf(m, fmaxf(fmaxf(fabsf(q.x), fabsf(q.y)), fmaxf(fabsf(q.z), fabsf(q.w))));
+            }
+            xs_exp = bf16_piece_scale(m);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const float4 q0 = has_piece ? xq[2 * i] : make_float4(0.f, 0.f, 0.f, 0.f);
+                const float4 q1 = has_piece ? xq[2 * i + 1] : make_float4(0.f, 0.f, 0.f, 0.f);
+                const float v[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
+                bf16_x_pairs(v, xs_exp, X + 4 * i);
             }
         }
         bool ok = true;
@@ -289,23 +333,45 @@ __global__ void __launch_bounds__(kThr, 1) decode1_kernel(const __grid_constant_
                 ok = false;
                 break;
             }
+            stamp_dep(a, l, 5 + j, lane == 0 && (warp == 0 || warp == 7), 0.f);
             const uint8_t *g0 = slot + sg.delta, *u0 = slot + a.up_off + su.delta;
-            for (int r = 0; r < n_gu; ++r) {
-                float gd = 0.f, ud = 0.f;
-                if (has_piece) {
-                    const uint8_t *gb = g0 + (size_t)r * rowB_gu + pb * kBlockBytes;
-                    const uint8_t *ub = u0 + (size_t)r * rowB_gu + pb * kBlockBytes;
-                    const float2 gsz = *reinterpret_cast<const float2 *>(gb);
-                    const float2 usz = *reinterpret_cast<const float2 *>(ub);
-                    uint32_t gw[8], uw[8];
-                    lds_words(gb + 8 + pq * 32, gw);
-                    lds_words(ub + 8 + pq * 32, uw);
-                    gd = finish_dot(nib64_fma(gw, xr), sx, gsz.x, gsz.y);
-                    ud = finish_dot(nib64_fma(uw, xr), sx, usz.x, usz.y);
+            for (int r0 = 0; r0 < n_gu; r0 += kGuRows) {
+                constexpr int kD = 2 * kGuRows;      // the group's dots: gate rows, then up rows
+                const uint8_t *pw[kD];
+                float2 sz[kD];
+                float acc[kD];
+                bool live[kD];
+#pragma unroll
+                for (int i = 0; i < kD; ++i) {
+                    const int r = r0 + (i % kGuRows);
+                    live[i] = has_piece && r < n_gu;
+                    const uint8_t *blk = (i < kGuRows ? g0 : u0) + (size_t)(live[i] ? r : 0) * rowB_gu +
+                                         (has_piece ? pb : 0) * kBlockBytes;
+                    sz[i] = live[i] ? *reinterpret_cast<const float2 *>(blk) : make_float2(0.f, 0.f);
+                    pw[i] = blk + 8 + pq * 32;
+                    acc[i] = 0.0f;
                 }
-                gd = warp_sum(gd);
-                ud = warp_sum(ud);
-                if (lane == 0) a.h[(size_t)j * Ip + gu_lo + r] = silu(gd) * ud;
+#pragma unroll
+                for (int wq = 0; wq < 4; ++wq) {      // 16 weights per step
+#pragma unroll
+                    for (int i = 0; i < kD; ++i) {
+                        const uint2 w = live[i] ? *reinterpret_cast<const uint2 *>(pw[i] + 8 * wq) : make_uint2(0u, 0u);
+                        acc[i] = nib8_dot_bf16(w.x, X + 8 * wq, acc[i]);
+                        acc[i] = nib8_dot_bf16(w.y, X + 8 * wq + 4, acc[i]);
+                    }
+                }
+                // partial = zero * sum(x) + scale * sum(q * x) over this lane's 64
+                float v[kD];
+#pragma unroll
+                for (int i = 0; i < kD; ++i)
+                    v[i] = live[i] ? fmaf(sz[i].x, scale2(acc[i], 133 - xs_exp), sz[i].y * sxp) : 0.f;
+                // lane l: total of value (l >> 2) & 7, i.e. gate row (l >> 2) for
+                // l < 16 and the matching up row 16 lanes higher
+                const float g = warp_sum_many<2 * kGuRows>(v);
+                const float u = __shfl_down_sync(0xffffffffu, g, 16);
+                const int i = lane >> 2;
+                if (lane < 16 && (lane & 3) == 0 && r0 + i < n_gu)
+                    a.h[(size_t)j * Ip + gu_lo + r0 + i] = silu(g) * u;
             }
         }
         if (__syncthreads_or(!ok || sh.abort)) break;
@@ -325,60 +391,85 @@ __global__ void __launch_bounds__(kThr, 1) decode1_kernel(const __grid_constant_
         if (__syncthreads_or(sh.abort)) break;
         stamp(a, l, 17);
 
-        float acc[kMaxDRows];
-#pragma unroll
-        for (int ri = 0; ri < kMaxDRows; ++ri) acc[ri] = 0.0f;
+        // this warp's weighted row sums, ysh[warp][ri], summed over its slots.
+        // Lane: piece pc (64 values of h, one quarter of a block) of row rs of
+        // each pass; P = Ip / 64 lanes per row, 32 / P rows per pass.
+        const int P = nbI * 4, RP = 32 / P;
+        const int pc = lane % P, rs = lane / P;
+        if (lane < kMaxDRows) ysh[warp * kMaxDRows + lane] = 0.0f;
         for (int j = warp; j < k && ok; j += kW) {
-            // this lane's h chunks (16 values each) and their even/odd sums
-            float2 hv[kMaxHChunks][8];
-            float2 hsum[kMaxHChunks];
+            // h of slot j -> the slot's gate/up part, consumed by now (zeros past
+            // I), then the lane's piece and its even/odd sums into registers
             const float *hj = a.h + (size_t)j * Ip;
+            float *hw = reinterpret_cast<float *>(slots + (size_t)j * a.slot_bytes);
+            {
+                // every load in flight before the first store (one L2 round trip)
+                float4 q4[kHLoads];
 #pragma unroll
-            for (int m = 0; m < kMaxHChunks; ++m) {
-                const int cc = lane + 32 * m;
-                const bool okc = cc * 16 < I;
-                hsum[m] = make_float2(0.f, 0.f);
-                float4 q4[4];
+                for (int q = 0; q < kHLoads; ++q) {
+                    const int i = lane + 32 * q;
+                    q4[q] = i < Ip / 4 && 4 * i < I ? __ldcg(reinterpret_cast<const float4 *>(hj) + i)
+                                                     : make_float4(0.f, 0.f, 0.f, 0.f);
+                }
+                // piece c (64 values) at 68 * c floats: the lanes' pieces start on
+                // distinct bank quads
 #pragma unroll
-                for (int v = 0; v < 4; ++v)
-                    q4[v] = okc ? __ldcg(reinterpret_cast<const float4 *>(hj + cc * 16) + v)
-                                : make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-                for (int v = 0; v < 4; ++v) {
-                    hv[m][2 * v] = make_float2(q4[v].x, q4[v].y);
-                    hv[m][2 * v + 1] = make_float2(q4[v].z, q4[v].w);
-                    hsum[m].x += q4[v].x + q4[v].z;
-                    hsum[m].y += q4[v].y + q4[v].w;
+                for (int q = 0; q < kHLoads; ++q) {
+                    const int i = lane + 32 * q;
+                    if (i < Ip / 4) reinterpret_cast<float4 *>(hw + (i >> 4) * 68)[i & 15] = q4[q];
                 }
             }
+            __syncwarp();
+            float2 hr[32];
+            float2 hs2 = make_float2(0.f, 0.f);
+            {
+                const float4 *hp = reinterpret_cast<const float4 *>(hw + pc * 68);
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    const float4 q = hp[i];
+                    hr[2 * i] = make_float2(q.x, q.y);
+                    hr[2 * i + 1] = make_float2(q.z, q.w);
+                    hs2.x += q.x + q.z;
+                    hs2.y += q.y + q.w;
+                }
+            }
+            __syncwarp();                              // the staging row is read; next slot may overwrite
+            stamp_dep(a, l, 21, lane == 0 && warp == 0, hs2.x);
             if (!(sh.hostmask >> j & 1u) && !wait_mbar_phase(wc, &sh.d_bar[j], par)) {
                 ok = false;
                 break;
             }
-            const uint8_t *d0 = slots + (size_t)j * a.slot_bytes + a.down_off + sd.delta;
+            stamp_dep(a, l, 22, lane == 0 && warp == 0, 0.f);
+            const uint8_t *d0 = slots + (size_t)j * a.slot_bytes + a.down_off + sd.delta +
+                                (pc >> 2) * kBlockBytes;                 // this lane's block of each row
             const float wj = sh.w[j];
+#pragma unroll 1
+            for (int p0 = 0; p0 * RP < n_d; p0 += 4) {      // four passes side by side
+                float v[4];
 #pragma unroll
-            for (int ri = 0; ri < kMaxDRows; ++ri) {
-                if (ri >= n_d) break;
-                const uint8_t *row = d0 + (size_t)ri * rowB_d;
+                for (int q = 0; q < 4; ++q) {
+                    const int ri = (p0 + q) * RP + rs;
+                    v[q] = 0.0f;
+                    if (ri < n_d) {
+                        const uint8_t *blk = d0 + (size_t)ri * rowB_d;
+                        const float2 sz = *reinterpret_cast<const float2 *>(blk);
+                        uint32_t wv[8];
+                        lds_words(blk + 8 + (pc & 3) * 32, wv);
+                        v[q] = finish_dot(nib64_fma(wv, hr), hs2, sz.x, sz.y);
+                    }
+                }
+                // sum over the P lanes of each row (contiguous, P a power of two)
 #pragma unroll
-                for (int m = 0; m < kMaxHChunks; ++m) {
-                    const int cc = lane + 32 * m;
-                    if (cc * 16 >= I) continue;
-                    const uint8_t *blk = row + (cc >> 4) * kBlockBytes;
-                    const float2 sz = *reinterpret_cast<const float2 *>(blk);
-                    const uint2 nv = *reinterpret_cast<const uint2 *>(blk + 8 + (cc & 15) * 8);
-                    const float part = finish_dot(nib16_fma(nv, hv[m]), hsum[m], sz.x, sz.y);
-                    acc[ri] = fmaf(wj, part, acc[ri]);
+                for (int q = 0; q < 4; ++q)
+                    for (int o = P >> 1; o > 0; o >>= 1) v[q] += __shfl_xor_sync(0xffffffffu, v[q], o);
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const int ri = (p0 + q) * RP + rs;
+                    if (pc == 0 && ri < n_d) ysh[warp * kMaxDRows + ri] += wj * v[q];
                 }
             }
         }
-#pragma unroll
-        for (int ri = 0; ri < kMaxDRows; ++ri) {
-            if (ri >= n_d) break;
-            const float v = warp_sum(acc[ri]);
-            if (lane == 0) ysh[warp * kMaxDRows + ri] = v;
-        }
+        stamp_dep(a, l, 23, lane == 0 && warp == 0, ysh[warp * kMaxDRows]);
         if (__syncthreads_or(!ok || sh.abort)) break;
         stamp(a, l, 19);
 
@@ -392,7 +483,7 @@ __global__ void __launch_bounds__(kThr, 1) decode1_kernel(const __grid_constant_
             if (a.y) a.y[(size_t)l * H + r] = y;
             if (a.y_bf16 && last) a.y_bf16[r] = float_to_bf16_bits(y);
             uint16_t *xo = last ? a.x_out : (a.xbuf ? a.xbuf + (size_t)((l + 1) & 1) * H : nullptr);
-            if (xo) xo[r] = float_to_bf16_bits(xs[xpad(r)] + y);
+            if (xo) xo[r] = float_to_bf16_bits(xs[xp4(r)] + y);
         }
         stamp(a, l, 20);
         if (l + 1 < a.L) {
@@ -461,6 +552,9 @@ hfq_status decode1_launch(const hfq4_layer *layers, int L, const float *logits, 
     const int G = sm_count();
     if (L < 1 || L > HFQ_MAX_STACK_LAYERS || k < 1 || k > kMaxK) return HFQ_ERR_UNSUPPORTED;
     if (expert_bytes(H, I) % 16) return HFQ_ERR_UNSUPPORTED;      // 16-byte aligned experts
+    if (x0_f32) return HFQ_ERR_UNSUPPORTED;     // the bf16 operands need bf16-valued activations
+    const int nbI_ = (I + kBlock - 1) / kBlock;
+    if (nbI_ != 1 && nbI_ != 2 && nbI_ != 4) return HFQ_ERR_UNSUPPORTED;   // 4 nbI lanes per down row
     if (H > kBlock * 8 || H % 8 || I > kBlock * 4 || I % 16 || E > HFQ_MAX_EXPERTS || E % 16)
         return HFQ_ERR_UNSUPPORTED;
     if ((H + G - 1) / G > kMaxDRows || (L > 1 && !xbuf) || !aligned16(x0) || (xbuf && !aligned16(xbuf)))
@@ -487,11 +581,14 @@ hfq_status decode1_launch(const hfq4_layer *layers, int L, const float *logits, 
     const size_t rowB_gu = (size_t)nbH * kBlockBytes, rowB_d = (size_t)nbI * kBlockBytes;
     const size_t gspan = up16((size_t)((I + G - 1) / G) * rowB_gu + 15);
     const size_t dspan = up16((size_t)((H + G - 1) / G) * rowB_d + 15);
-    const size_t slot = (2 * gspan + dspan + 127) / 128 * 128;
+    // the gate/up part of a slot also stages the slot's h in the down phase:
+    // 4 nbI pieces of 64 floats, 68 apart
+    const size_t gu_part = std::max(2 * gspan, up16((size_t)nbI * 4 * 68 * 4));
+    const size_t slot = (gu_part + dspan + 127) / 128 * 128;
     size_t off = (size_t)k * slot;
-    a.slot_bytes = (int)slot; a.up_off = (int)gspan; a.down_off = (int)(2 * gspan);
+    a.slot_bytes = (int)slot; a.up_off = (int)gspan; a.down_off = (int)gu_part;
     a.xs_off = (int)off;
-    off += up16((Hp + 2 * (Hp >> 6)) * 4);
+    off += up16((Hp + 4 * (Hp >> 6)) * 4);
     a.ptab_off = (int)off;
     off += (size_t)2 * E * 8;
     a.ltab_stride = (int)up16((size_t)E);

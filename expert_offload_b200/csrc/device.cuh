@@ -20,6 +20,33 @@ __device__ __forceinline__ float warp_sum(float v)
     return v;
 }
 
+// Sums each of V values (V a power of two, 2 <= V <= 32) over the 32 lanes
+// with V - 1 + log2(32 / V) shuffles, in a chain five shuffles deep: at each
+// of the first log2 V steps a lane keeps half of its values and adds its
+// partner's copy of them.  Returns, in lane l, the total of value
+// (l >> (5 - log2 V)) & (V - 1).  `a` is overwritten.
+template <int V>
+__device__ __forceinline__ float warp_sum_many(float (&a)[V])
+{
+    static_assert(V >= 2 && V <= 32 && (V & (V - 1)) == 0, "V: a power of two in [2, 32]");
+    const int lane = threadIdx.x & 31;
+    int m = 16;
+#pragma unroll
+    for (int n = V; n > 1; n >>= 1, m >>= 1) {
+        const bool up = (lane & m) != 0;
+#pragma unroll
+        for (int i = 0; i < n / 2; ++i) {
+            const float send = up ? a[i] : a[i + n / 2];
+            const float keep = up ? a[i + n / 2] : a[i];
+            a[i] = keep + __shfl_xor_sync(0xffffffffu, send, m);
+        }
+    }
+    float v = a[0];
+#pragma unroll
+    for (int mm = 32 / V / 2; mm > 0; mm >>= 1) v += __shfl_xor_sync(0xffffffffu, v, mm);
+    return v;
+}
+
 __device__ __forceinline__ float bf16_bits_to_float(uint16_t b)
 {
     return __uint_as_float(((uint32_t)b) << 16);

@@ -102,16 +102,21 @@ def up16(b):
     return (b + 15) // 16 * 16
 
 
+def xp4(c):
+    return c + 4 * (c >> 6)
+
+
 def decode1_layout(H, I, E, k, G):
     nbH, nbI = -(-H // 256), -(-I // 256)
     Hp = nbH * 256
     rowB_gu, rowB_d = nbH * K_BB, nbI * K_BB
     gspan = up16(-(-I // G) * rowB_gu + 15)
     dspan = up16(-(-H // G) * rowB_d + 15)
-    slot = (2 * gspan + dspan + 127) // 128 * 128
+    gu_part = max(2 * gspan, up16(nbI * 4 * 68 * 4))     # also stages h: pieces of 64 floats, 68 apart
+    slot = (gu_part + dspan + 127) // 128 * 128
     off = k * slot
-    lay = dict(slot=slot, up=gspan, down=2 * gspan, gspan=gspan, dspan=dspan, xs=off)
-    off += up16((Hp + 2 * (Hp >> 6)) * 4)
+    lay = dict(slot=slot, up=gspan, down=gu_part, gspan=gspan, dspan=dspan, xs=off)
+    off += up16((Hp + 4 * (Hp >> 6)) * 4)
     lay["ptab"] = off
     off += 2 * E * 8
     lay["ltab_stride"] = up16(E)
@@ -126,11 +131,12 @@ def decode1_layout(H, I, E, k, G):
 
 def decode1_accepts(H, I, E, k, G):
     return (1 <= k <= 16 and H <= 2048 and H % 8 == 0 and I <= 1024 and I % 16 == 0
+            and -(-I // 256) in (1, 2, 4)
             and E <= 512 and E % 16 == 0 and -(-H // G) <= D1_MAX_DROWS)
 
 
 @pytest.mark.parametrize("H,I,E,k,G", [(2048, 512, 256, 8, 148), (2048, 512, 512, 8, 148),
-                                       (256, 128, 16, 4, 148), (2048, 768, 128, 8, 148),
+                                       (256, 128, 16, 4, 148), (2048, 1024, 128, 8, 148),
                                        (2048, 512, 256, 16, 148), (1024, 1024, 64, 6, 132)])
 def test_decode1_copies_and_reads_stay_in_their_slot(H, I, E, k, G):
     assert decode1_accepts(H, I, E, k, G)
@@ -159,9 +165,38 @@ def test_decode1_copies_and_reads_stay_in_their_slot(H, I, E, k, G):
             # reads: rows r < n, blocks of 136 bytes, within the copied span
             last = delta + (n - 1) * rowB + rowB
             assert last <= ln
-    # the next slot starts after the largest span set
-    assert 2 * lay["gspan"] + lay["dspan"] <= lay["slot"]
-    assert lay["xs"] + up16((nbH * 256 + 2 * (nbH * 256 >> 6)) * 4) <= lay["ptab"]
+    # the next slot starts after the largest span set; h fits the gate/up part
+    assert lay["down"] >= 2 * lay["gspan"] and lay["down"] + lay["dspan"] <= lay["slot"]
+    assert nbI * 4 * 68 * 4 <= lay["down"]
+    # staged h pieces: 16-byte aligned, quarter-warps on distinct bank quads
+    for q0 in range(0, 32, 8):
+        starts = {((lane % (nbI * 4)) * 68) % 32 for lane in range(q0, q0 + 8)}
+        assert len(starts) == min(8, nbI * 4)
+    assert lay["xs"] + up16((nbH * 256 + 4 * (nbH * 256 >> 6)) * 4) <= lay["ptab"]
+    # x: f32 at column xp4(c); lanes read 64-wide slices with 16-byte loads
+    Hp = nbH * 256
+    for lane in range(32):
+        pb, pq = lane >> 2, lane & 3
+        if pb >= nbH:
+            continue
+        c0 = pb * 256 + pq * 64
+        assert (lay["xs"] + 4 * xp4(c0)) % 16 == 0
+        for i in range(64):
+            assert xp4(c0 + i) == xp4(c0) + i                 # slice contiguous
+        assert xp4(c0 + 63) < Hp + 4 * (Hp >> 6)
+    # down phase: lane piece pc of row rs reads its block's scale/zero and 32
+    # payload bytes; P lanes per row tile the warp
+    P = nbI * 4
+    assert 32 % P == 0
+    for lane in range(32):
+        pc = lane % P
+        for ri in range(D1_MAX_DROWS):
+            off = ri * rowB_d + (pc >> 2) * K_BB
+            assert off + 8 + (pc & 3) * 32 + 32 <= D1_MAX_DROWS * rowB_d
+    # quarter-warps of 16-byte loads hit distinct bank quads
+    for q0 in range(0, 32, 8):
+        starts = {xp4((l >> 2) * 256 + (l & 3) * 64) % 32 for l in range(q0, q0 + 8) if (l >> 2) < nbH}
+        assert len(starts) == len([l for l in range(q0, q0 + 8) if (l >> 2) < nbH])
 
 
 def test_decode1_declines_shapes_outside_its_registers():
@@ -169,3 +204,4 @@ def test_decode1_declines_shapes_outside_its_registers():
     assert not decode1_accepts(2048, 2048, 256, 8, 148)     # two 16-value h chunks per lane
     assert not decode1_accepts(2048, 512, 256, 17, 148)     # two slots per warp
     assert not decode1_accepts(2048, 512, 250, 8, 148)      # 16-byte table copies
+    assert not decode1_accepts(2048, 768, 128, 8, 148)      # 12 lanes per down row do not tile a warp
