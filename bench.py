@@ -36,8 +36,8 @@ def parse():
     ap.add_argument("--steps", type=int, default=10000)
     ap.add_argument("--warmup", type=int, default=50)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=["decode", "verify", "offload"], default="decode")
-    ap.add_argument("--tokens", type=int, default=8, help="tokens per step (verify)")
+    ap.add_argument("--workload", choices=["decode", "verify", "offload", "prefill"], default="decode")
+    ap.add_argument("--tokens", type=int, default=8, help="tokens per step (verify, prefill)")
     ap.add_argument("--resident-layers", type=int, default=None, help="offload: N")
     ap.add_argument("--hot", type=int, default=0, help="offload: hot experts per host layer")
     ap.add_argument("--hbm-read-probe", action="store_true")
@@ -350,7 +350,8 @@ def run_ours(args, rank, world, local_rank):
         "gpu_launches": launches_per_step * K,
         "clocks": clocks,
     }
-    kernel = ("stack_kernel (persistent: all layers of one step per launch)"
+    kernel = (("decode1_kernel" if T == 1 else "stack_kernel") +
+              " (persistent: all layers of one step per launch)"
               if launches_per_step == 1 else "per-layer route + gate/up + down launches")
     if args.workload == "offload":
         pcie = measure_pcie(torch, eo)
@@ -393,6 +394,102 @@ def run_ours(args, rank, world, local_rank):
         dist.barrier()
         graphs.clear()
         dist.destroy_process_group()
+    store.close()
+    return out
+
+
+# ------------------------------------------------------------- prefill arm
+
+def run_prefill(args):
+    """One prefill chunk through one MoE layer (512 experts, Zipf(1.1) expert
+    popularity): a step routes T tokens with grouping by expert (moe_route)
+    and runs hfq4_moe_forward, on the tensor-core path (the default for
+    T > 8) and, for comparison, on the GEMV path.  Each step routes a
+    different chunk of tokens (distinct logits and activations cycled)."""
+    import numpy as np
+    import torch
+
+    import expert_offload_b200 as eo
+    import synth
+    from expert_offload_b200.model import ExpertStore
+    from synth import workloads as W
+
+    torch.cuda.set_device(0)
+    w = W.WORKLOADS[4]
+    H, I, E, k, T = w.hidden, w.inter, w.experts, w.top_k, args.tokens
+    G = max(2, min(args.distinct_tokens, 8))
+
+    def fill(l, g, u, d):
+        s = torch.cuda.current_stream().cuda_stream
+        synth.weights_dev(g.data_ptr(), w.seed, l, 0, E, synth.MAT_GATE, I, H, W.WEIGHT_SIGMA, s)
+        synth.weights_dev(u.data_ptr(), w.seed, l, 0, E, synth.MAT_UP, I, H, W.WEIGHT_SIGMA, s)
+        synth.weights_dev(d.data_ptr(), w.seed, l, 0, E, synth.MAT_DOWN, H, I, W.WEIGHT_SIGMA, s)
+
+    store = ExpertStore(torch, 1, E, H, I, fill)
+    logits = torch.from_numpy(np.stack([W.zipf_logits(w, 0, g * T, T) for g in range(G)])).cuda()
+    xs = torch.from_numpy(np.stack([W.activations(w, g * T, T)[0] for g in range(G)]).view(np.int16)).cuda()
+    idx = torch.empty((T, k), dtype=torch.int32, device="cuda")
+    wts = torch.empty((T, k), dtype=torch.float32, device="cuda")
+    cnt = torch.empty(E, dtype=torch.int32, device="cuda")
+    off = torch.empty(E + 1, dtype=torch.int32, device="cuda")
+    perm = torch.empty(T * k, dtype=torch.int32, device="cuda")
+    rws = torch.zeros(max(256, eo.hfq_route_workspace_bytes(T, E, k)), dtype=torch.uint8, device="cuda")
+    y = torch.empty((T, H), dtype=torch.float32, device="cuda")
+    need = eo.hfq4_moe_workspace_bytes(T, k, H, I, E)
+    ws = torch.zeros(need, dtype=torch.uint8, device="cuda")
+    # 256 MB written between steps flushes the 126 MB L2 (weights of a chunk are < 1 GB)
+    flush = torch.empty(256 * 2**20, dtype=torch.uint8, device="cuda")
+    stream = torch.cuda.Stream()
+
+    def step(g, path):
+        eo.moe_route(logits[g], T, E, k, idx, wts, cnt, off, perm, rws, stream=stream)
+        eo.hfq4_moe_forward(store.layers[0], xs[g], eo.HFQ_BF16, T, idx, wts, k, y, ws, cnt=cnt,
+                            off=off, perm=perm, path=path, stream=stream)
+
+    def timed(path, steps):
+        with torch.cuda.stream(stream):
+            for i in range(args.warmup):
+                step(i % G, path)
+            torch.cuda.synchronize()
+            ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                  for _ in range(steps)]
+            for i in range(steps):
+                flush.fill_(i & 0xFF)
+                ev[i][0].record(stream)
+                step(i % G, path)
+                ev[i][1].record(stream)
+            torch.cuda.synchronize()
+        eo.hfq_workspace_status(ws, stream)
+        return sum(a.elapsed_time(b) for a, b in ev) / steps
+
+    sampler = ClockSampler(0)
+    sampler.start()
+    ms_tc = timed(eo.PATH_AUTO, args.steps)
+    clocks = sampler.stop()
+    ms_gemv = timed(eo.PATH_GEMV, max(3, min(args.steps, 20)))
+    used = int((cnt > 0).sum().item())
+    eb = eo.hfq4_expert_bytes(H, I)
+    flops = 2.0 * T * k * 3 * H * I
+    d = json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json"))) if os.path.exists(
+        os.path.join(ROOT, "MEASURED_PEAKS.json")) else {"bf16_tflops": 1590.0}
+    peak = float(d["bf16_tflops"])
+    achieved = flops / (ms_tc / 1e3) / 1e12
+    out = {"metric": METRIC, "value": round(T / (ms_tc / 1e3), 1), "unit": "tokens/s", "n_gpus": 1,
+           "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_tc, 5),
+           "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+           "data": "synthetic",
+           "config": {"workload": w.name, "tokens": T, "layers": 1, "hidden": H, "inter": I,
+                      "experts": E, "top_k": k, "path": "tcgen05 grouped dequant-to-bf16 GEMM",
+                      "experts_used": used, "expert_bytes": used * eb,
+                      "l2": "256 MB written between timed steps",
+                      "gemv_path_ms_per_step": round(ms_gemv, 4),
+                      "gemv_path_tokens_per_s": round(T / (ms_gemv / 1e3), 1)},
+           "gpu_launches": 1 + 5, "clocks": clocks,
+           "roofline": {"bound": "tensor", "achieved": round(achieved, 1), "peak": peak,
+                        "unit": "TFLOP/s", "frac": round(achieved / peak, 4), "traffic": None,
+                        "flops_per_step": flops,
+                        "hbm_time_floor_ms": round(used * eb / 6522.1e9 * 1e3, 4),
+                        "peak_source": "measured bf16 burst"}}
     store.close()
     return out
 
@@ -511,6 +608,10 @@ def main():
         if rank != 0:
             return
         print(json.dumps(run_reference(args)), flush=True)
+        return
+    if args.workload == "prefill":
+        if rank == 0:
+            print(json.dumps(run_prefill(args)), flush=True)
         return
     out = run_ours(args, rank, world, local_rank)
     if rank == 0:
