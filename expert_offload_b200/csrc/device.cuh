@@ -101,6 +101,14 @@ hfq_status decode1_launch(const hfq4_layer *layers, int L, const float *logits, 
                           uint16_t *xbuf, float *h, float *y, uint16_t *y_bf16, int32_t *idx_all,
                           float *wts_all, unsigned *ctl, long long timeout_ns, int extra_arrivals,
                           cudaStream_t s);
+// Persistent decode kernel for 2..8 tokens (verify.cu); launch_stack hands such
+// batches to it when verify_launch accepts the shape (else HFQ_ERR_UNSUPPORTED
+// with no launch, and the general kernel runs).
+hfq_status verify_launch(const hfq4_layer *layers, int L, const float *logits, const int32_t *idx_in,
+                         const float *wts_in, const void *x0, bool x0_f32, int T, int k, uint16_t *x_out,
+                         uint16_t *xbuf, float *h, float *y, uint16_t *y_bf16, int32_t *idx_all,
+                         float *wts_all, unsigned *ctl, long long timeout_ns, int extra_arrivals,
+                         cudaStream_t s);
 int sm_count();
 
 // Tensor-core expert path (tc.cu).

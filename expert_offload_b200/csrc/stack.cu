@@ -857,6 +857,10 @@ hfq_status launch_stack(const hfq4_layer *layers, int L, const float *logits, co
                                              h, y, y_bf16, idx_all, wts_all, ctl, timeout_ns,
                                              extra_arrivals, s);
         if (st != HFQ_ERR_UNSUPPORTED) return st;
+    } else {
+        const hfq_status st = verify_launch(layers, L, logits, idx_in, wts_in, x0, x0_f32, T, k, x_out, xbuf,
+                                            h, y, y_bf16, idx_all, wts_all, ctl, timeout_ns, extra_arrivals, s);
+        if (st != HFQ_ERR_UNSUPPORTED) return st;
     }
     StackArgs a;
     memset(&a, 0, sizeof a);
