@@ -1,6 +1,6 @@
 // verify.cu - persistent decode kernel for 2..8 tokens per step (speculative
 // verify batches): every MoE layer of a step in one cooperative launch, one
-// CTA of eight consumer warps and one producer warp per SM.
+// CTA of eight consumer warps and four producer warps per SM.
 //
 // hipfire thread, "HFQ quantisation format and GEMV": decode is a GEMV over
 // 136-byte blocks, bound by the bytes of the selected experts; with T tokens a
@@ -12,10 +12,12 @@
 //      warp 0 lists the unique experts (ascending) and their (expert, token)
 //      pairs; all threads turn the T inputs into per-64-value pieces of
 //      scaled bf16 pairs (gemv.cuh);
-//   2. the producer warp streams one item per ring stage with 1-D bulk copies
+//   2. the producer warps stream one item per ring stage with 1-D bulk copies
 //      (TMA, no multicast): the gate/up share of every unique expert, then its
 //      down share; host-mapped experts are read with 16-byte loads (hipfire
-//      offload explainer, "PCIe pass-through");
+//      offload explainer, "PCIe pass-through").  Items go round-robin to four
+//      producer warps: one warp's consecutive bulk copies issue slowly while
+//      many are in flight, several warps' copies overlap;
 //   3. consumer warp w takes the pairs p = w, w + 8, ... : for a gate/up item
 //      it computes all of the CTA's rows of its token at once (8 dots in
 //      flight, one batched warp reduction) and writes h = silu(g) * u;
@@ -39,7 +41,8 @@ namespace hfq {
 namespace {
 
 constexpr int kCW = 8;                  // consumer warps
-constexpr int kThr = (kCW + 1) * 32;    // + the producer warp
+constexpr int kPW = 4;                  // producer warps: stage s is filled by producer s % kPW
+constexpr int kThr = (kCW + kPW) * 32;
 constexpr int kMaxT = 8;
 constexpr int kMaxP = 64;               // (expert, token) pairs per layer: T * k <= 64
 constexpr int kMaxU = 64;
@@ -70,6 +73,7 @@ struct VArgs {
     int extra_arrivals;       // test hook: grid barriers wait for this many more CTAs
     int NS, stage_bytes;      // ring
     int xp_off, xres_off, ysh_off, hst_off, sh_off;
+    unsigned long long *timeline;   // debug: [G][L][32] %globaltimer stamps, or null
 };
 
 struct VShared {
@@ -89,6 +93,7 @@ struct VShared {
     float pw[kMaxP];            // routing weight of pair p
     const uint8_t *ubase[kMaxU];
     unsigned char uloc[kMaxU];
+    int armed_seq[kMaxNS];      // latest item sequence number armed in each stage, or -1
     int abort;
     int last_cta;
 };
@@ -108,6 +113,24 @@ __device__ __forceinline__ Span span_of(size_t off, size_t len)
     s.len = len ? (int)(e16 - a16) : 0;
     s.delta = (int)(off - a16);
     return s;
+}
+
+// Debug timeline: stamp s of layer l for this CTA (ns of %globaltimer).
+__device__ __forceinline__ void vstamp(const VArgs &a, int l, int s, bool who)
+{
+    if (a.timeline && who && l < a.L)
+        a.timeline[((size_t)blockIdx.x * a.L + l) * 32 + s] = globaltimer_ns();
+}
+
+// Debug: where a bounded wait of this kernel gave up, recorded once per
+// launch into control words 3..5 (site, layer, item sequence) when the status
+// word shows a timeout.
+__device__ __forceinline__ void note_wait(const VArgs &a, bool ok, int site, int l, int seq)
+{
+    if (!ok && atomicCAS(a.ctl + 3, 0u, (unsigned)site) == 0u) {
+        a.ctl[4] = (unsigned)l;
+        a.ctl[5] = (unsigned)seq;
+    }
 }
 
 __device__ __forceinline__ void consumer_sync() { asm volatile("bar.sync 1, %0;" ::"r"(kCW * 32) : "memory"); }
@@ -177,21 +200,33 @@ __device__ void build_pairs(VShared &sh, const VArgs &a, int l)
         sh.ubase[u] = static_cast<const uint8_t *>(a.eptr[l][e]);
         sh.uloc[u] = a.eloc[l] ? a.eloc[l][e] : 0;
     }
-    if (lane == 0) {
-        int n = 0;
-        for (int u = 0; u < U; ++u) {
-            sh.pair0[u] = n;
-            for (unsigned m = sh.umask[u]; m; m &= m - 1u) {
+    // pairs: lane u (then u + 32) writes expert u's pairs at its prefix offset
+    int run = 0;
+    for (int u0 = 0; u0 < kMaxU; u0 += 32) {
+        const int u = u0 + lane;
+        const int n = u < U ? __popc(sh.umask[u]) : 0;
+        int inc = n;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int v = __shfl_up_sync(0xffffffffu, inc, o);
+            if (lane >= o) inc += v;
+        }
+        int q = run + inc - n;
+        if (u < U) {
+            sh.pair0[u] = q;
+            for (unsigned m = sh.umask[u]; m; m &= m - 1u, ++q) {
                 const int t = __ffs(m) - 1, j = sh.ujt[u][t];
-                sh.pt[n] = t;
-                sh.prow[n] = t * k + j;
-                sh.pw[n] = sh.wsel[t][j];
-                ++n;
+                sh.pt[q] = t;
+                sh.prow[q] = t * k + j;
+                sh.pw[q] = sh.wsel[t][j];
             }
         }
-        sh.pair0[U] = n;
+        run += __shfl_sync(0xffffffffu, inc, 31);
+    }
+    if (lane == 0) {
+        sh.pair0[U] = run;
         sh.U = U;
-        sh.P = n;
+        sh.P = run;
     }
     __syncwarp();
 }
@@ -226,6 +261,7 @@ __global__ void __launch_bounds__(kThr, 1) verify_kernel(const __grid_constant__
         for (int s = 0; s < kMaxNS; ++s) {
             mbar_init(&sh.full[s], 1);
             mbar_init(&sh.empty[s], kCW);
+            sh.armed_seq[s] = -1;
         }
         sh.abort = 0;
         fence_mbar_init();
@@ -233,8 +269,8 @@ __global__ void __launch_bounds__(kThr, 1) verify_kernel(const __grid_constant__
     __syncthreads();
 
     int stage_base = 0;                 // ring items of earlier layers (same in every warp)
-    int issued = 0;                     // producer: items issued so far (all layers)
     for (int l = 0; l < a.L; ++l) {
+        vstamp(a, l, 0, tid == 0);
         // ---------------------------------------------- 1. route, pairs, inputs
         if (warp < T) {
             if (a.idx_in) {
@@ -260,12 +296,20 @@ __global__ void __launch_bounds__(kThr, 1) verify_kernel(const __grid_constant__
         {
             // layer input: token t, values 8*tid .. 8*tid+7 (Hp/8 <= 256 groups)
             const uint16_t *xin = l == 0 ? a.x0 : a.xbuf + (size_t)(l & 1) * T * H;
-            for (int t = 0; t < T && warp < kCW; ++t) {
+            uint4 xq[kMaxT];                      // every token's 8 values in flight at once
+#pragma unroll
+            for (int t = 0; t < kMaxT; ++t)
+                xq[t] = (t < T && warp < kCW && 8 * tid < H)
+                            ? __ldcg(reinterpret_cast<const uint4 *>(xin + (size_t)t * H) + tid)
+                            : make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+            for (int t = 0; t < kMaxT; ++t) {
+                if (t >= T || warp >= kCW) break;
                 float v[8];
 #pragma unroll
                 for (int i = 0; i < 8; ++i) v[i] = 0.0f;
                 if (8 * tid < H) {
-                    const uint4 q = __ldcg(reinterpret_cast<const uint4 *>(xin + (size_t)t * H) + tid);
+                    const uint4 q = xq[t];
                     const uint32_t w4[4] = {q.x, q.y, q.z, q.w};
 #pragma unroll
                     for (int r = 0; r < 4; ++r) {
@@ -284,32 +328,39 @@ __global__ void __launch_bounds__(kThr, 1) verify_kernel(const __grid_constant__
                 for (int i = tid; i < kCW * T * kMaxDRows; i += kCW * 32) ysh[i] = 0.0f;
         }
         __syncthreads();
+        vstamp(a, l, 1, tid == 0);
         if (warp == 0) build_pairs(sh, a, l);
         if (__syncthreads_or(sh.abort)) break;
+        vstamp(a, l, 2, tid == 0);
         const int U = sh.U, P = sh.P;
         if (a.idx_all && c == 0 && warp < T && lane < k) {
             a.idx_all[((size_t)l * T + warp) * k + lane] = sh.sel[warp][lane];
             a.wts_all[((size_t)l * T + warp) * k + lane] = sh.wsel[warp][lane];
         }
 
-        if (warp == kCW) {
-            // ------------------------------------------ 2. producer warp
+        if (warp >= kCW) {
+            // ------------------------------------------ 2. producer warps
             for (int i = 0; i < 2 * U && !sh.abort; ++i) {
                 const int seq = stage_base + i, s = seq % NS, u = i < U ? i : i - U;
+                // a stage always has the same producer: its uses are armed in order
+                if (s % kPW != warp - kCW) continue;
                 if (seq >= NS) {
                     int ok = 1;
-                    if (lane == 0) ok = wait_mbar_phase(wc, &sh.empty[s], ((seq / NS) - 1) & 1) ? 1 : 0;
+                    if (lane == 0) {
+                        ok = wait_mbar_phase(wc, &sh.empty[s], ((seq / NS) - 1) & 1) ? 1 : 0;
+                        note_wait(a, ok, 1, l, seq);
+                    }
                     if (!__shfl_sync(0xffffffffu, ok, 0)) break;
                 }
-                // the stage was last read by the generic proxy (consumers, released
-                // through the empty barrier)
-                fence_proxy_async_smem();
+                // the stage's last readers released it through the empty barrier,
+                // which this wait acquired: the bulk copy may overwrite it
                 const uint8_t *base = sh.ubase[u];
                 if (((uintptr_t)base & 15u) != 0) {               // bulk copies start on 16 bytes
                     if (lane == 0) { atomicCAS(a.ctl, 0u, (unsigned)HFQ_ERR_ARG); sh.abort = 1; }
                     break;
                 }
                 uint8_t *st = ring + (size_t)s * a.stage_bytes;
+                if (lane == 0) sh.armed_seq[s] = seq;
                 if (!sh.uloc[u]) {
                     if (lane == 0) {
                         if (i < U) {
@@ -340,8 +391,10 @@ __global__ void __launch_bounds__(kThr, 1) verify_kernel(const __grid_constant__
                     __syncwarp();
                     if (lane == 0) mbar_arrive(&sh.full[s]);
                 }
-                issued = seq + 1;
+                vstamp(a, l, 8, lane == 0 && i == U - 1);
+                vstamp(a, l, 10 + i, lane == 0 && i < 10);
             }
+            vstamp(a, l, 9, lane == 0 && warp == kCW);
         } else {
             // ------------------------------------------ 3. gate/up items
             const int pb = lane >> 2, pq = lane & 3;
@@ -350,16 +403,20 @@ __global__ void __launch_bounds__(kThr, 1) verify_kernel(const __grid_constant__
             for (int u = 0; u < U; ++u) {
                 const int seq = stage_base + u, s = seq % NS;
                 const uint8_t *st = ring + (size_t)s * a.stage_bytes;
-                int p = sh.pair0[u] + ((warp - sh.pair0[u]) % kCW + kCW) % kCW;
-                bool waited = false;
-                for (; p < sh.pair0[u + 1] && ok; p += kCW) {
-                    if (!waited) {
-                        int w = 1;
-                        if (lane == 0) w = wait_mbar_phase(wc, &sh.full[s], (seq / NS) & 1) ? 1 : 0;
-                        ok = __shfl_sync(0xffffffffu, w, 0) != 0;
-                        waited = true;
-                        if (!ok) break;
+                // every warp waits for the item before it releases the stage, with
+                // or without pairs in it: an arrival on the empty barrier of a use
+                // that is not armed yet would count toward the previous use
+                if (ok) {
+                    int w = 1;
+                    if (lane == 0) {
+                        w = wait_mbar_phase(wc, &sh.full[s], (seq / NS) & 1) ? 1 : 0;
+                        note_wait(a, w, 2, l, seq);
                     }
+                    ok = __shfl_sync(0xffffffffu, w, 0) != 0;
+                    vstamp(a, l, 3, lane == 0 && u == 0 && warp == 0);
+                }
+                int p = sh.pair0[u] + ((warp - sh.pair0[u]) % kCW + kCW) % kCW;
+                for (; p < sh.pair0[u + 1] && ok; p += kCW) {
                     uint32_t X[32];
                     int xe = 0;
                     float sxp = 0.0f;
@@ -374,6 +431,7 @@ __global__ void __launch_bounds__(kThr, 1) verify_kernel(const __grid_constant__
                         xe = (int)es.x;
                         sxp = __uint_as_float(es.y);
                     }
+                    vstamp(a, l, 24, lane == 0 && warp == 0 && p == 0);
                     float *hrow = a.h + (size_t)sh.prow[p] * Ip + gu_lo;
                     const uint8_t *g0 = st + sg.delta, *u0 = st + up_off + su.delta;
                     for (int r0 = 0; r0 < n_gu; r0 += kGuRows) {
@@ -414,6 +472,7 @@ __global__ void __launch_bounds__(kThr, 1) verify_kernel(const __grid_constant__
                         const int i = lane >> 2;
                         if (lane < 16 && (lane & 3) == 0 && r0 + i < n_gu) hrow[r0 + i] = silu(g) * uu;
                     }
+                    vstamp(a, l, 25, lane == 0 && warp == 0 && p == 0);
                 }
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&sh.empty[s]);        // this warp is done with the stage
@@ -421,13 +480,18 @@ __global__ void __launch_bounds__(kThr, 1) verify_kernel(const __grid_constant__
             // ------------------------------------------ 4. h exchange
             unsigned *hcnt = a.ctl + kCtlH + (size_t)l * kCtlHStride;
             consumer_sync();
+            vstamp(a, l, 4, tid == 0);
             if (tid == 0) {
                 if (!ok) sh.abort = 1;
                 __threadfence();
                 red_release_gpu_add(hcnt, 1u);
-                if (!sh.abort && !wait_counter_ge(wc, hcnt, (unsigned)G)) sh.abort = 1;
+                if (!sh.abort && !wait_counter_ge(wc, hcnt, (unsigned)G)) {
+                    sh.abort = 1;
+                    note_wait(a, false, 3, l, 0);
+                }
             }
             consumer_sync();
+            vstamp(a, l, 5, tid == 0);
             ok = ok && !sh.abort;
 
             // ------------------------------------------ 5. down items
@@ -455,6 +519,17 @@ __global__ void __launch_bounds__(kThr, 1) verify_kernel(const __grid_constant__
                 const int seq = stage_base + U + u, s = seq % NS;
                 const uint8_t *st = ring + (size_t)s * a.stage_bytes;
                 bool waited = false;
+                if (ok && pnext >= sh.pair0[u + 1]) {
+                    // no pair of this warp in the item: still wait for it before
+                    // releasing the stage (see the gate/up loop)
+                    int w = 1;
+                    if (lane == 0) {
+                        w = wait_mbar_phase(wc, &sh.full[s], (seq / NS) & 1) ? 1 : 0;
+                        note_wait(a, w, 4, l, seq);
+                    }
+                    ok = __shfl_sync(0xffffffffu, w, 0) != 0;
+                    waited = true;
+                }
                 while (ok && pnext < sh.pair0[u + 1]) {
                     const int p = pnext;
                     float *hw = hw0 + (size_t)buf * Pl * kHStride;
@@ -479,28 +554,32 @@ __global__ void __launch_bounds__(kThr, 1) verify_kernel(const __grid_constant__
                     }
                     if (!waited) {
                         int w = 1;
-                        if (lane == 0) w = wait_mbar_phase(wc, &sh.full[s], (seq / NS) & 1) ? 1 : 0;
+                        if (lane == 0) {
+                            w = wait_mbar_phase(wc, &sh.full[s], (seq / NS) & 1) ? 1 : 0;
+                            note_wait(a, w, 4, l, seq);
+                        }
                         ok = __shfl_sync(0xffffffffu, w, 0) != 0;
                         waited = true;
                         if (!ok) break;
                     }
+                    vstamp(a, l, 26, lane == 0 && warp == 0 && p == 0);
                     const uint8_t *d0 = st + sd.delta + (pc >> 2) * kBlockBytes;   // this lane's block of each row
                     const float wp = sh.pw[p];
                     float *yt = ysh + ((size_t)warp * T + sh.pt[p]) * kMaxDRows;
 #pragma unroll 1
                     for (int p0 = 0; p0 * RP < n_d; p0 += 4) {      // four passes side by side
+                        // rows past n_d repeat the last row (inside the span; their
+                        // sums are dropped) so the four passes run side by side
+                        // without a branch
                         float v[4];
 #pragma unroll
                         for (int q = 0; q < 4; ++q) {
-                            const int ri = (p0 + q) * RP + rs;
-                            v[q] = 0.0f;
-                            if (ri < n_d) {
-                                const uint8_t *blk = d0 + (size_t)ri * rowB_d;
-                                const float2 sz = *reinterpret_cast<const float2 *>(blk);
-                                uint32_t wv[8];
-                                lds_words(blk + 8 + (pc & 3) * 32, wv);
-                                v[q] = finish_dot(nib64_fma(wv, hr), hs2, sz.x, sz.y);
-                            }
+                            const int ri = min((p0 + q) * RP + rs, n_d - 1);
+                            const uint8_t *blk = d0 + (size_t)ri * rowB_d;
+                            const float2 sz = *reinterpret_cast<const float2 *>(blk);
+                            uint32_t wv[8];
+                            lds_words(blk + 8 + (pc & 3) * 32, wv);
+                            v[q] = finish_dot(nib64_fma(wv, hr), hs2, sz.x, sz.y);
                         }
 #pragma unroll
                         for (int q = 0; q < 4; ++q)
@@ -511,6 +590,7 @@ __global__ void __launch_bounds__(kThr, 1) verify_kernel(const __grid_constant__
                             if (pc == 0 && ri < n_d) yt[ri] += wp * v[q];
                         }
                     }
+                    vstamp(a, l, 27, lane == 0 && warp == 0 && p == 0);
                 }
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&sh.empty[s]);
@@ -520,6 +600,7 @@ __global__ void __launch_bounds__(kThr, 1) verify_kernel(const __grid_constant__
         }
         stage_base += 2 * U;
         __syncthreads();
+        vstamp(a, l, 6, tid == 0);
 
         // ---------------------------------------------- 6. combine, residual
         if (!sh.abort && tid < T * n_d) {
@@ -534,25 +615,30 @@ __global__ void __launch_bounds__(kThr, 1) verify_kernel(const __grid_constant__
             uint16_t *xo = last ? a.x_out : (a.xbuf ? a.xbuf + (size_t)((l + 1) & 1) * T * H : nullptr);
             if (xo) xo[o] = float_to_bf16_bits(xres[t * kMaxDRows + ri] + y);
         }
+        vstamp(a, l, 7, tid == 0);
         if (l + 1 < a.L) {
             __syncthreads();
             if (tid == 0) {
                 unsigned *bar = a.ctl + kCtlBar + l;
                 __threadfence();
                 red_release_gpu_add(bar, 1u);
-                if (!sh.abort && !wait_counter_ge(wc, bar, (unsigned)(G + a.extra_arrivals))) sh.abort = 1;
+                if (!sh.abort && !wait_counter_ge(wc, bar, (unsigned)(G + a.extra_arrivals))) {
+                    sh.abort = 1;
+                    note_wait(a, false, 5, l, 0);
+                }
             }
             if (__syncthreads_or(sh.abort)) break;
         }
     }
 
-    // no copy may still be writing this CTA's shared memory when it exits: the
-    // last NS issued items' phases complete (bounded)
+    // no copy may still be writing this CTA's shared memory when it exits:
+    // every stage's last armed phase completes (bounded)
     __syncthreads();
-    if (warp == kCW && lane == 0) {
-        for (int seq = max(0, issued - NS); seq < issued; ++seq) {
+    if (tid < NS) {
+        const int seq = sh.armed_seq[tid];
+        if (seq >= 0) {
             const uint64_t t0 = globaltimer_ns();
-            while (!mbar_try_wait(&sh.full[seq % NS], (seq / NS) & 1) && !deadline_passed(t0, a.timeout_ns)) {
+            while (!mbar_try_wait(&sh.full[tid], (seq / NS) & 1) && !deadline_passed(t0, a.timeout_ns)) {
             }
         }
     }
@@ -614,6 +700,7 @@ hfq_status verify_launch(const hfq4_layer *layers, int L, const float *logits, c
     a.x0 = static_cast<const uint16_t *>(x0); a.x_out = x_out; a.xbuf = xbuf; a.h = h; a.y = y;
     a.y_bf16 = y_bf16; a.idx_all = idx_all; a.wts_all = wts_all;
     a.ctl = ctl; a.timeout_ns = timeout_ns; a.extra_arrivals = extra_arrivals;
+    a.timeline = static_cast<unsigned long long *>(option_timeline());
     a.L = L; a.T = T; a.E = E; a.k = k; a.H = H; a.I = I;
 
     // shared-memory layout: ring stages, then the fixed parts

@@ -245,12 +245,17 @@ hfq_status hfq4_moe_forward_noalloc(const hfq4_layer *layer, const void *x, hfq_
  *     persistent-kernel launch makes its grid barriers wait for this many
  *     CTAs that do not exist, so the wait runs out without any fault.
  *   HFQ_OPT_TIMELINE_BUFFER: debug; the device address of a u64 buffer of
- *     2 * n_layers * 32 words, zero-filled (0 = off).  Persistent-kernel
- *     launches then write %globaltimer stamps (ns) for two CTAs (CTA 0 and CTA
- *     gridDim/2), per layer: [0] layer start, [1] routed, [2] table built,
- *     [3 + s] ring stage s ready (s < 12), [16] gate/up done, [17] all h
- *     ready, [18] h staged, [19] down done, [20] layer end, [21] all copies
- *     issued, [22 + s] bytes of stage s landed (s < 10, one token only).
+ *     n_sms * n_layers * 32 words, zero-filled (0 = off).  Persistent-kernel
+ *     launches then write %globaltimer stamps (ns), per layer l at word
+ *     (row * n_layers + l) * 32 + s.  The one-token and general kernels write
+ *     rows 0 and 1 (CTA 0 and CTA gridDim/2): [0] layer start, [1] routed,
+ *     [2] table built, [3 + s] ring stage s ready (s < 12), [16] gate/up done,
+ *     [17] all h ready, [18] h staged, [19] down done, [20] layer end, [21]
+ *     all copies issued, [22 + s] bytes of stage s landed (s < 10).  The
+ *     2..8-token kernel writes row c for every CTA c: [0] layer start, [1]
+ *     inputs and routing done, [2] pair table built, [3] first gate/up item
+ *     landed, [4] gate/up done, [5] h exchange done, [6] down done, [7]
+ *     outputs written, [8] last gate/up item issued, [9] all items issued.
  * Returns HFQ_ERR_ARG for an unknown option or a value out of range.
  */
 #define HFQ_OPT_WAIT_TIMEOUT_NS 1
