@@ -350,7 +350,7 @@ def run_ours(args, rank, world, local_rank):
         "gpu_launches": launches_per_step * K,
         "clocks": clocks,
     }
-    kernel = (("decode1_kernel" if T == 1 else "stack_kernel") +
+    kernel = (("decode1_kernel" if T == 1 else "verify_kernel") +
               " (persistent: all layers of one step per launch)"
               if launches_per_step == 1 else "per-layer route + gate/up + down launches")
     if args.workload == "offload":
@@ -378,8 +378,14 @@ def run_ours(args, rank, world, local_rank):
                            "mean_launch_ms": round(mean_launch_ms, 5)}
     else:
         achieved = bytes_per_step / (mean_launch_ms / 1e3) / 1e9
+        # DRAM bytes (read + write) of decode1_kernel from an ncu capture of the
+        # first 10 layers of this workload (133.84 MB read + 5.02 MB written),
+        # scaled by 4 to the 40-layer launch (the per-layer work is the same)
+        traffic = (133.8368e6 + 5.0196e6) * 4 if (args.workload == "decode" and T == 1
+                                                 and L == 40 and not args.layers) else None
         out["roofline"] = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak,
-                           "unit": "GB/s", "frac": round(achieved / peak, 4), "traffic": None,
+                           "unit": "GB/s", "frac": round(achieved / peak, 4), "traffic": traffic,
+                           "traffic_unit": "DRAM bytes per launch",
                            "peak_source": peak_kind, "kernel": kernel,
                            "bytes_per_launch": round(bytes_per_step),
                            "mean_launch_ms": round(mean_launch_ms, 5)}

@@ -75,9 +75,11 @@ struct WsHeader {
 constexpr size_t kWsHeader = sizeof(WsHeader);   // 256 bytes
 
 // Control block at the head of a persistent kernel's workspace, in 32-bit
-// words: [0] status (the WsHeader word), [1] CTAs finished, [64 + l] grid
-// barrier after layer l, [128 + 128 l] CTAs whose h rows of layer l are
-// written.  Zero between launches: the last CTA of a launch clears what it used.
+// words: [0] status (the WsHeader word), [1] CTAs finished, [3..5] debug: the
+// first bounded wait of the 2..8-token kernel that gave up (site, layer, item),
+// [64 + l] grid barrier after layer l, [128 + 128 l] CTAs whose h rows of layer
+// l are written.  Zero between launches: the last CTA of a launch clears what
+// it used (a wait that gave up leaves its record until the status is read).
 constexpr int kCtlDone = 1, kCtlBar = 64, kCtlH = 128, kCtlHStride = 128;
 constexpr size_t kCtlWords = kCtlH + (size_t)HFQ_MAX_STACK_LAYERS * kCtlHStride;
 constexpr size_t kCtlBytes = (kCtlWords * 4 + 255) / 256 * 256;
