@@ -117,7 +117,16 @@ __global__ void __launch_bounds__(kTcThr, 1) tc_kernel(const __grid_constant__ T
     uint32_t chunk = 0;                              // stages used so far (buffer = chunk & 1)
     const int total = a.item_off[a.E];
 
-    for (int item = blockIdx.x; item < total; item += gridDim.x) {
+    // this thread's weight row (gate/up: one matrix; down: half of each K
+    // chunk) and activation pieces; the next chunk's loads (of this item or,
+    // at its last chunk, of the next item) are in flight while a chunk is
+    // dequantised and multiplied
+    const int row = tid & (kM - 1), which = tid >> 7;
+    struct Geo {
+        int p0, nvalid, r0;
+        const uint8_t *rrow;
+    };
+    auto geo_of = [&](int item) {
         int lo = 0, hi = a.E;                        // item_off[lo] <= item < item_off[lo + 1]
         while (hi - lo > 1) {
             const int mid = (lo + hi) >> 1;
@@ -125,39 +134,69 @@ __global__ void __launch_bounds__(kTcThr, 1) tc_kernel(const __grid_constant__ T
         }
         const int e = lo, local = item - a.item_off[e];
         const int rt = local % rtiles, nt = local / rtiles;
-        const int p0 = a.off[e] + nt * kN, nvalid = min(kN, a.cnt[e] - nt * kN);
-        const int r0 = rt * kM;
+        Geo g;
+        g.p0 = a.off[e] + nt * kN;
+        g.nvalid = min(kN, a.cnt[e] - nt * kN);
+        g.r0 = rt * kM;
         const uint8_t *base = static_cast<const uint8_t *>(a.eptr[e]);
-        const uint8_t *A0 = GU ? base : base + 2 * mg;       // gate (or down)
-        const uint8_t *A1 = base + mg;                       // up
+        const uint8_t *A = GU ? (which ? base + mg : base) : base + 2 * mg;   // gate / up, or down
+        g.rrow = A + (size_t)(g.r0 + row) * rowB;
+        return g;
+    };
+    float2 nsz;
+    uint2 nw[4];
+    uint4 nx[(kN * kKC / 8) / kTcThr];
+    auto load = [&](const Geo &g, int kc2) {
+        const int blk = (kc2 * kKC) / kBlock, sub = ((kc2 * kKC) % kBlock) / 2;   // nibble byte
+        const uint8_t *rp = g.rrow + (size_t)blk * kBlockBytes;
+        nsz = __ldg(reinterpret_cast<const float2 *>(rp));
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+            if (GU || i < 2) nw[i] = __ldg(reinterpret_cast<const uint2 *>(rp + 8 + sub + (GU ? 0 : 16 * which) + 8 * i));
+#pragma unroll
+        for (int i = 0; i < (kN * kKC / 8) / kTcThr; ++i) {
+            const int id = tid + i * kTcThr;
+            const int n = id & (kN - 1), k8 = id >> 7;
+            nx[i] = n < g.nvalid ? __ldg(reinterpret_cast<const uint4 *>(a.xin + (size_t)(g.p0 + n) * K + kc2 * kKC + k8 * 8))
+                                 : make_uint4(0u, 0u, 0u, 0u);
+        }
+    };
+    Geo cur{};
+    if ((int)blockIdx.x < total) {
+        cur = geo_of(blockIdx.x);
+        load(cur, 0);
+    }
+    for (int item = blockIdx.x; item < total; item += gridDim.x) {
+        const Geo g = cur;
+        const int p0 = g.p0, nvalid = g.nvalid, r0 = g.r0;
+        const int next = item + (int)gridDim.x;
+        Geo ng{};
+        if (next < total) ng = geo_of(next);
 
         for (int kc = 0; kc < nK; ++kc, ++chunk) {
             const int s = chunk & 1;
             uint8_t *st = smem + (size_t)s * kOps * kTileBytes;
-            if (commits[s] && !abort) tc_wait(a, &mma_bar[s], (commits[s] - 1) & 1, abort);
-            const int blk = (kc * kKC) / kBlock, sub = ((kc * kKC) % kBlock) / 2;   // nibble byte
+            const float2 sz = nsz;
+            uint2 w[4];
+            uint4 xv[(kN * kKC / 8) / kTcThr];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) w[i] = nw[i];
+#pragma unroll
+            for (int i = 0; i < (kN * kKC / 8) / kTcThr; ++i) xv[i] = nx[i];
             if (!abort) {
-                // weights: each thread one row (gate/up) or half a row (down)
-                const int row = GU ? (tid & (kM - 1)) : (tid & (kM - 1));
-                const int which = tid >> 7;                  // gate/up: matrix; down: K half
-                const uint8_t *A = (GU && which) ? A1 : A0;
-                const uint8_t *rp = A + (size_t)(r0 + row) * rowB + (size_t)blk * kBlockBytes;
-                const float2 sz = __ldg(reinterpret_cast<const float2 *>(rp));
+                if (kc + 1 < nK) load(g, kc + 1);
+                else if (next < total) load(ng, 0);
+            }
+            if (commits[s] && !abort) tc_wait(a, &mma_bar[s], (commits[s] - 1) & 1, abort);
+            if (!abort) {
                 uint8_t *dst = st + (GU && which ? kTileBytes : 0);
                 if (GU) {
-                    uint2 w[4];
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) w[i] = __ldg(reinterpret_cast<const uint2 *>(rp + 8 + sub + 8 * i));
 #pragma unroll
                     for (int i = 0; i < 4; ++i) {
                         *reinterpret_cast<uint4 *>(dst + tile_off(row, 2 * i)) = deq8(w[i].x, sz.x, sz.y);
                         *reinterpret_cast<uint4 *>(dst + tile_off(row, 2 * i + 1)) = deq8(w[i].y, sz.x, sz.y);
                     }
                 } else {
-                    uint2 w[2];
-#pragma unroll
-                    for (int i = 0; i < 2; ++i)
-                        w[i] = __ldg(reinterpret_cast<const uint2 *>(rp + 8 + sub + 16 * which + 8 * i));
 #pragma unroll
                     for (int i = 0; i < 2; ++i) {
                         *reinterpret_cast<uint4 *>(dst + tile_off(row, 4 * which + 2 * i)) = deq8(w[i].x, sz.x, sz.y);
@@ -170,10 +209,7 @@ __global__ void __launch_bounds__(kTcThr, 1) tc_kernel(const __grid_constant__ T
                 for (int i = 0; i < (kN * kKC / 8) / kTcThr; ++i) {
                     const int id = tid + i * kTcThr;
                     const int n = id & (kN - 1), k8 = id >> 7;
-                    uint4 v = make_uint4(0u, 0u, 0u, 0u);
-                    if (n < nvalid)
-                        v = __ldg(reinterpret_cast<const uint4 *>(a.xin + (size_t)(p0 + n) * K + kc * kKC + k8 * 8));
-                    *reinterpret_cast<uint4 *>(bt + tile_off(n, k8)) = v;
+                    *reinterpret_cast<uint4 *>(bt + tile_off(n, k8)) = xv[i];
                 }
             }
             fence_proxy_async_smem();
@@ -226,6 +262,7 @@ __global__ void __launch_bounds__(kTcThr, 1) tc_kernel(const __grid_constant__ T
         tc_fence_before_sync();
         __syncthreads();
         if (s_abort) abort = 1;
+        cur = ng;
     }
     // no MMA may still write tensor memory when it is freed
     if (tid == 0 && chunk) {
