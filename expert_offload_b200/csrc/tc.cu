@@ -4,8 +4,8 @@
 // Per expert e with T_e routed (token, slot) pairs (grouped by moe_route):
 //   G = X_e Wg^T, U = X_e Wu^T   (bf16 x bf16 -> f32 in tensor memory)
 //   H_e = bf16(silu(G) * U)
-//   O = H_e Wd^T                  (bf16 x bf16 -> f32)
-//   y[t] += w_tj * O[pair]        (f32 atomic adds)
+//   O = H_e Wd^T                  (bf16 x bf16 -> f32), one row per pair
+//   y[t] = sum_j w_tj * O[pair (t, j)]   (slot order: deterministic)
 // The weights are dequantised from HFQ4 straight into shared memory as bf16,
 // RN_bf16(fmaf(scale, q, zero)), in the canonical K-major no-swizzle layout
 // the MMA reads (8-row x 16-byte core matrices).  Prior art on the pages: the
@@ -33,7 +33,7 @@ struct TcArgs {
     const float *wts;              // [T*k] routing weights, flat
     const uint16_t *xin;           // gate/up: X_perm [T*k][H]; down: H_perm [T*k][I] (bf16)
     uint16_t *hout;                // gate/up: H_perm out
-    float *y;                      // down: y [T][H], accumulated
+    float *o;                      // down: O [T*k][H] f32, row q = pair perm[q]
     const int32_t *item_off;       // [E+1] prefix of work items of this phase
     unsigned *status;
     long long timeout_ns;
@@ -253,8 +253,7 @@ __global__ void __launch_bounds__(kTcThr, 1) tc_kernel(const __grid_constant__ T
                     if (GU) {
                         a.hout[(size_t)p * a.I + r0 + r] = float_to_bf16_bits(silu(g[j]) * u[j]);
                     } else {
-                        const int pe = a.perm[p];
-                        atomicAdd(a.y + (size_t)(pe / a.k) * a.H + r0 + r, a.wts[pe] * g[j]);
+                        a.o[(size_t)p * a.H + r0 + r] = g[j];
                     }
                 }
             }
@@ -298,14 +297,16 @@ __global__ void tc_plan_kernel(const int32_t *__restrict__ cnt, int E, int I, in
     }
 }
 
-// X_perm[q] = x[token of pair perm[q]] as bf16 (16 bytes per thread step).
+// X_perm[q] = x[token of pair perm[q]] as bf16 (16 bytes per thread step);
+// pos[perm[q]] = q.
 __global__ void tc_gather_kernel(const void *__restrict__ x, int x_f32, const int32_t *__restrict__ perm,
-                                 int P, int k, int H, uint16_t *__restrict__ xp)
+                                 int P, int k, int H, uint16_t *__restrict__ xp, int32_t *__restrict__ pos)
 {
     const size_t n8 = (size_t)P * H / 8;
     for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n8;
          i += (size_t)gridDim.x * blockDim.x) {
         const size_t q = i / (H / 8), c = (i - q * (H / 8)) * 8;
+        if (c == 0) pos[perm[q]] = (int32_t)q;
         const size_t src = (size_t)(perm[q] / k) * H + c;
         uint4 v;
         if (x_f32) {
@@ -323,11 +324,32 @@ __global__ void tc_gather_kernel(const void *__restrict__ x, int x_f32, const in
     }
 }
 
-__global__ void tc_y_bf16_kernel(const float *__restrict__ y, size_t n, uint16_t *__restrict__ yb)
+// y[t][r] = sum over slots j (in order) of w[t*k + j] * O[pos[t*k + j]][r],
+// four rows per thread step; optional bf16 copy.
+__global__ void tc_combine_kernel(const float *__restrict__ o, const int32_t *__restrict__ pos,
+                                  const float *__restrict__ wts, int T, int k, int H, float *__restrict__ y,
+                                  uint16_t *__restrict__ yb)
 {
-    for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
-         i += (size_t)gridDim.x * blockDim.x)
-        yb[i] = float_to_bf16_bits(y[i]);
+    const size_t n4 = (size_t)T * H / 4;
+    for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n4;
+         i += (size_t)gridDim.x * blockDim.x) {
+        const size_t t = i / (H / 4), c = (i - t * (H / 4)) * 4;
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int j = 0; j < k; ++j) {
+            const float w = wts[t * k + j];
+            const float4 v = __ldg(reinterpret_cast<const float4 *>(o + (size_t)pos[t * k + j] * H + c));
+            acc.x = fmaf(w, v.x, acc.x);
+            acc.y = fmaf(w, v.y, acc.y);
+            acc.z = fmaf(w, v.z, acc.z);
+            acc.w = fmaf(w, v.w, acc.w);
+        }
+        *reinterpret_cast<float4 *>(y + t * H + c) = acc;
+        if (yb) {
+            const uint32_t lo = float_to_bf16_bits(acc.x) | ((uint32_t)float_to_bf16_bits(acc.y) << 16);
+            const uint32_t hi = float_to_bf16_bits(acc.z) | ((uint32_t)float_to_bf16_bits(acc.w) << 16);
+            *reinterpret_cast<uint2 *>(yb + t * H + c) = make_uint2(lo, hi);
+        }
+    }
 }
 
 int tc_sms()
@@ -347,7 +369,7 @@ size_t tc_workspace_bytes(int T, int k, int H, int I, int E)
 {
     const size_t P = (size_t)T * k;
     auto r256 = [](size_t b) { return (b + 255) / 256 * 256; };
-    return r256(P * H * 2) + r256(P * I * 2) + 2 * r256((size_t)(E + 1) * 4);
+    return r256(P * H * 2) + r256(P * I * 2) + 2 * r256((size_t)(E + 1) * 4) + r256(P * H * 4) + r256(P * 4);
 }
 
 bool tc_supported(int H, int I)
@@ -371,6 +393,10 @@ hfq_status launch_tc(const hfq4_layer &L, const void *x, bool x_f32, int T, int 
     int32_t *gu_off = reinterpret_cast<int32_t *>(w);
     w += r256((size_t)(E + 1) * 4);
     int32_t *dn_off = reinterpret_cast<int32_t *>(w);
+    w += r256((size_t)(E + 1) * 4);
+    float *ob = reinterpret_cast<float *>(w);
+    w += r256(P * H * 4);
+    int32_t *pos = reinterpret_cast<int32_t *>(w);
 
     static bool attr = false;
     const int smem_gu = 2 * 3 * kTileBytes, smem_dn = 2 * 2 * kTileBytes;
@@ -382,20 +408,17 @@ hfq_status launch_tc(const hfq4_layer &L, const void *x, bool x_f32, int T, int 
     tc_plan_kernel<<<1, 512, 0, s>>>(cnt, E, I, H, gu_off, dn_off);
     const size_t n8 = P * H / 8;
     tc_gather_kernel<<<(unsigned)std::min<size_t>((n8 + 255) / 256, (size_t)tc_sms() * 16), 256, 0, s>>>(
-        x, x_f32 ? 1 : 0, perm, (int)P, k, H, xp);
-    cudaMemsetAsync(y, 0, (size_t)T * H * sizeof(float), s);
+        x, x_f32 ? 1 : 0, perm, (int)P, k, H, xp, pos);
     TcArgs a;
     a.eptr = L.expert_ptr; a.cnt = cnt; a.off = off; a.perm = perm; a.wts = wts;
     a.status = status; a.timeout_ns = timeout_ns; a.E = E; a.H = H; a.I = I; a.k = k;
-    a.xin = xp; a.hout = hp; a.y = nullptr; a.item_off = gu_off;
+    a.xin = xp; a.hout = hp; a.o = nullptr; a.item_off = gu_off;
     tc_kernel<true><<<tc_sms(), kTcThr, smem_gu, s>>>(a);
-    a.xin = hp; a.hout = nullptr; a.y = y; a.item_off = dn_off;
+    a.xin = hp; a.hout = nullptr; a.o = ob; a.item_off = dn_off;
     tc_kernel<false><<<tc_sms(), kTcThr, smem_dn, s>>>(a);
-    if (y_bf16) {
-        const size_t n = (size_t)T * H;
-        tc_y_bf16_kernel<<<(unsigned)std::min<size_t>((n + 255) / 256, (size_t)tc_sms() * 16), 256, 0, s>>>(
-            y, n, y_bf16);
-    }
+    const size_t n4 = (size_t)T * H / 4;
+    tc_combine_kernel<<<(unsigned)std::min<size_t>((n4 + 255) / 256, (size_t)tc_sms() * 16), 256, 0, s>>>(
+        ob, pos, wts, T, k, H, y, y_bf16);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return fail(HFQ_ERR_CUDA, "tensor-core path launch: %s", cudaGetErrorString(e));
     return HFQ_OK;

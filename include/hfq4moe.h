@@ -172,8 +172,9 @@ typedef struct {
  *           tensor cores.  GEMV forces CUDA cores; TC forces the tensor-core
  *           path [WMMA]: weights dequantised to RN_bf16(fmaf(scale, q, zero)),
  *           x rounded to bf16 (exact for bf16 input), f32 accumulation, h
- *           rounded to bf16 before the down projection, y accumulated with f32
- *           atomic adds (the order of the k slots is not fixed).
+ *           rounded to bf16 before the down projection, each pair's down
+ *           output kept in f32 and y summed over the k slots in slot order
+ *           (deterministic).
  *   y:      f32 [T][H] out.  y_bf16: optional bf16 [T][H] out (NULL = none).
  *   workspace: hfq4_moe_workspace_bytes(T, k, H, I, E) bytes of device
  *           scratch (plus the same again for HFQ_PATH_TC with T <= 8),
