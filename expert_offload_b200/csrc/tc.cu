@@ -20,9 +20,11 @@ namespace {
 
 constexpr int kM = 128;                    // weight rows per tile (MMA M)
 constexpr int kN = 128;                    // token pairs per tile (MMA N)
-constexpr int kKC = 64;                    // K per pipeline stage (4 MMAs of K = 16)
+constexpr int kKC = 128;                   // K per pipeline stage (8 MMAs of K = 16)
+constexpr int kWGU = kKC / 16;             // 8-byte nibble words per row and chunk (gate/up)
+constexpr int kWD = kKC / 32;              // per half row (down: two threads per row)
 constexpr int kTcThr = 256;                // 8 warps
-constexpr int kTileBytes = kM * kKC * 2;   // one 128 x 64 bf16 operand tile (16 KB)
+constexpr int kTileBytes = kM * kKC * 2;   // one 128 x kKC bf16 operand tile
 constexpr uint32_t kLbo = (kM / 8) * 128;  // bytes between 8-element K chunks (2048)
 constexpr uint32_t kSbo = 128;             // bytes between 8-row groups
 constexpr uint32_t kTmemCols = 256;
@@ -144,15 +146,16 @@ __global__ void __launch_bounds__(kTcThr, 1) tc_kernel(const __grid_constant__ T
         return g;
     };
     float2 nsz;
-    uint2 nw[4];
+    uint2 nw[kWGU];
     uint4 nx[(kN * kKC / 8) / kTcThr];
     auto load = [&](const Geo &g, int kc2) {
         const int blk = (kc2 * kKC) / kBlock, sub = ((kc2 * kKC) % kBlock) / 2;   // nibble byte
         const uint8_t *rp = g.rrow + (size_t)blk * kBlockBytes;
         nsz = __ldg(reinterpret_cast<const float2 *>(rp));
 #pragma unroll
-        for (int i = 0; i < 4; ++i)
-            if (GU || i < 2) nw[i] = __ldg(reinterpret_cast<const uint2 *>(rp + 8 + sub + (GU ? 0 : 16 * which) + 8 * i));
+        for (int i = 0; i < kWGU; ++i)
+            if (GU || i < kWD)
+                nw[i] = __ldg(reinterpret_cast<const uint2 *>(rp + 8 + sub + (GU ? 0 : 8 * kWD * which) + 8 * i));
 #pragma unroll
         for (int i = 0; i < (kN * kKC / 8) / kTcThr; ++i) {
             const int id = tid + i * kTcThr;
@@ -177,10 +180,10 @@ __global__ void __launch_bounds__(kTcThr, 1) tc_kernel(const __grid_constant__ T
             const int s = chunk & 1;
             uint8_t *st = smem + (size_t)s * kOps * kTileBytes;
             const float2 sz = nsz;
-            uint2 w[4];
+            uint2 w[kWGU];
             uint4 xv[(kN * kKC / 8) / kTcThr];
 #pragma unroll
-            for (int i = 0; i < 4; ++i) w[i] = nw[i];
+            for (int i = 0; i < kWGU; ++i) w[i] = nw[i];
 #pragma unroll
             for (int i = 0; i < (kN * kKC / 8) / kTcThr; ++i) xv[i] = nx[i];
             if (!abort) {
@@ -192,15 +195,15 @@ __global__ void __launch_bounds__(kTcThr, 1) tc_kernel(const __grid_constant__ T
                 uint8_t *dst = st + (GU && which ? kTileBytes : 0);
                 if (GU) {
 #pragma unroll
-                    for (int i = 0; i < 4; ++i) {
+                    for (int i = 0; i < kWGU; ++i) {
                         *reinterpret_cast<uint4 *>(dst + tile_off(row, 2 * i)) = deq8(w[i].x, sz.x, sz.y);
                         *reinterpret_cast<uint4 *>(dst + tile_off(row, 2 * i + 1)) = deq8(w[i].y, sz.x, sz.y);
                     }
                 } else {
 #pragma unroll
-                    for (int i = 0; i < 2; ++i) {
-                        *reinterpret_cast<uint4 *>(dst + tile_off(row, 4 * which + 2 * i)) = deq8(w[i].x, sz.x, sz.y);
-                        *reinterpret_cast<uint4 *>(dst + tile_off(row, 4 * which + 2 * i + 1)) = deq8(w[i].y, sz.x, sz.y);
+                    for (int i = 0; i < kWD; ++i) {
+                        *reinterpret_cast<uint4 *>(dst + tile_off(row, 2 * kWD * which + 2 * i)) = deq8(w[i].x, sz.x, sz.y);
+                        *reinterpret_cast<uint4 *>(dst + tile_off(row, 2 * kWD * which + 2 * i + 1)) = deq8(w[i].y, sz.x, sz.y);
                     }
                 }
                 // activations: 128 token rows x 64 values, 16 bytes per piece
