@@ -221,7 +221,7 @@ __device__ void warp_topk(const float *__restrict__ row, int E, int k, int *sel,
     const int lane = threadIdx.x & 31;
     int my_e;
     float my_w;
-    warp_topk_lane<M>(row, E, k, my_e, my_w);
+    warp_topk_rounds<M>(row, E, k, my_e, my_w, [](int, int) {});
     if (lane < k) {
         if (ubase) {
             ubase[lane] = static_cast<const uint8_t *>(eptr[my_e]);

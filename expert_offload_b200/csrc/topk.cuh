@@ -21,12 +21,18 @@ __device__ __forceinline__ float key_value(uint32_t k)
     return __uint_as_float((k & 0x80000000u) ? (k & 0x7fffffffu) : ~k);
 }
 
-// Lane i holds experts i*M .. i*M+M-1 of `row` (E logits); k rounds of a warp
-// max over the lanes' best keys, the lowest lane winning ties, which is the
-// lowest expert index.  Lane j < k returns the j-th selected expert and its
-// weight exp(v_j - v_0) / sum_i<k exp(v_i - v_0); other lanes return e = -1.
-template <int M>
-__device__ void warp_topk_lane(const float *__restrict__ row, int E, int k, int &my_e, float &my_w)
+// Lane i holds experts i*M .. i*M+M-1 of `row` (E logits) and keeps its three
+// largest untaken keys in registers (k0 >= k1 >= k2; equal keys in expert
+// order).  Each of the k rounds takes the warp max of the lanes' k0, the
+// lowest lane winning ties (the lowest expert index); the winner shifts its
+// cache (selects, no branch) and, once three of its keys are taken, rescans
+// its M keys on a warp-uniform branch.  `on_round(j, e)` runs on the whole
+// warp right after round j has selected expert e.  Lane j < k returns the
+// j-th selected expert and its weight exp(v_j - v_0) / sum_i<k exp(v_i - v_0);
+// other lanes return e = -1.
+template <int M, class F>
+__device__ __forceinline__ void warp_topk_rounds(const float *__restrict__ row, int E, int k, int &my_e,
+                                                 float &my_w, F &&on_round)
 {
     const int lane = threadIdx.x & 31;
     uint32_t key[M];
@@ -35,43 +41,72 @@ __device__ void warp_topk_lane(const float *__restrict__ row, int E, int k, int 
         const int e = lane * M + i;
         key[i] = e < E ? order_key(__ldg(row + e)) : 0u;
     }
-    uint32_t taken = 0, bk = key[0];
-    int bi = 0;
+    uint32_t k0, k1, k2;
+    int i0, i1, i2;
+    auto top3 = [&](uint32_t taken) {
+        k0 = k1 = k2 = 0u;
+        i0 = i1 = i2 = 0;
 #pragma unroll
-    for (int i = 1; i < M; ++i)
-        if (key[i] > bk) { bk = key[i]; bi = i; }
+        for (int i = 0; i < M; ++i) {
+            const uint32_t x = (taken >> i & 1u) ? 0u : key[i];
+            const bool g0 = x > k0, g1 = x > k1, g2 = x > k2;
+            k2 = g1 ? k1 : (g2 ? x : k2);
+            i2 = g1 ? i1 : (g2 ? i : i2);
+            k1 = g0 ? k0 : (g1 ? x : k1);
+            i1 = g0 ? i0 : (g1 ? i : i1);
+            k0 = g0 ? x : k0;
+            i0 = g0 ? i : i0;
+        }
+    };
+    top3(0u);
+    uint32_t taken = 0u;
+    int wins = 0;
     float v0 = 0.0f, s = 0.0f, my_ex = 0.0f;
     my_e = -1;
     for (int j = 0; j < k; ++j) {
-        const uint32_t m = __reduce_max_sync(0xffffffffu, bk);
-        const unsigned ball = __ballot_sync(0xffffffffu, bk == m);
+        const uint32_t m = __reduce_max_sync(0xffffffffu, k0);
+        const unsigned ball = __ballot_sync(0xffffffffu, k0 == m);
         const int win = __ffs(ball) - 1;
-        const int e = __shfl_sync(0xffffffffu, lane * M + bi, win);
+        const int e = __shfl_sync(0xffffffffu, lane * M + i0, win);
+        const bool won = lane == win;
+        taken |= won ? 1u << i0 : 0u;
+        k0 = won ? k1 : k0;
+        i0 = won ? i1 : i0;
+        k1 = won ? k2 : k1;
+        i1 = won ? i2 : i1;
+        k2 = won ? 0u : k2;
+        wins += won ? 1 : 0;
+        if (M > 3 && __any_sync(0xffffffffu, won && wins == 3)) {
+            if (won) {
+                top3(taken);
+                wins = 0;
+            }
+        }
         const float v = key_value(m);
         if (j == 0) v0 = v;
         const float ex = __expf(v - v0);
         s += ex;
         if (lane == j) { my_ex = ex; my_e = e; }
-        if (lane == win) {
-            taken |= 1u << bi;
-            bool any = false;
-            bk = 0u; bi = 0;
-#pragma unroll
-            for (int i = 0; i < M; ++i)
-                if (!(taken >> i & 1u) && (!any || key[i] > bk)) { bk = key[i]; bi = i; any = true; }
-        }
+        on_round(j, e);
     }
     my_w = my_ex / s;
 }
 
-// warp_topk_lane with M chosen from E (E <= 512).
+// warp_topk_rounds with M chosen from E (E <= 512).
+template <class F>
+__device__ __forceinline__ void warp_route_rounds(const float *row, int E, int k, int &my_e, float &my_w,
+                                                  F &&on_round)
+{
+    if (E <= 32) warp_topk_rounds<1>(row, E, k, my_e, my_w, on_round);
+    else if (E <= 64) warp_topk_rounds<2>(row, E, k, my_e, my_w, on_round);
+    else if (E <= 128) warp_topk_rounds<4>(row, E, k, my_e, my_w, on_round);
+    else if (E <= 256) warp_topk_rounds<8>(row, E, k, my_e, my_w, on_round);
+    else warp_topk_rounds<16>(row, E, k, my_e, my_w, on_round);
+}
+
 __device__ __forceinline__ void warp_route(const float *row, int E, int k, int &my_e, float &my_w)
 {
-    if (E <= 32) warp_topk_lane<1>(row, E, k, my_e, my_w);
-    else if (E <= 64) warp_topk_lane<2>(row, E, k, my_e, my_w);
-    else if (E <= 128) warp_topk_lane<4>(row, E, k, my_e, my_w);
-    else if (E <= 256) warp_topk_lane<8>(row, E, k, my_e, my_w);
-    else warp_topk_lane<16>(row, E, k, my_e, my_w);
+    warp_route_rounds(row, E, k, my_e, my_w, [](int, int) {});
 }
 
 }  // namespace hfq
