@@ -3,6 +3,7 @@
 #include <cfloat>
 
 #include "device.cuh"
+#include "topk.cuh"
 
 namespace hfq {
 namespace {
@@ -101,67 +102,28 @@ __global__ void dequant_kernel(const uint8_t *__restrict__ blocks, int rows, int
 }
 
 // ------------------------------------------------------------------- route
-// One CTA per token (hipfire offload explainer, opening section: top-8 of a
-// layer's experts).  k rounds of a CTA-wide argmax over (logit, -index).
-constexpr int kRouteThreads = 256;
+// One warp per token (hipfire offload explainer, opening section: top-8 of a
+// layer's experts): the k largest logits, ties to the lower expert index, and
+// their softmax renormalised over the selected k (topk.cuh).
+constexpr int kRouteWarps = 4;
 
-__device__ __forceinline__ bool better(float a, int ia, float b, int ib)
-{
-    return a > b || (a == b && ia < ib);
-}
-
-__global__ void __launch_bounds__(kRouteThreads)
-route_kernel(const float *__restrict__ logits, int E, int k, int32_t *__restrict__ idx,
+__global__ void __launch_bounds__(kRouteWarps * 32)
+route_kernel(const float *__restrict__ logits, int T, int E, int k, int32_t *__restrict__ idx,
              float *__restrict__ wts)
 {
-    __shared__ float sl[HFQ_MAX_EXPERTS];
-    __shared__ unsigned char taken[HFQ_MAX_EXPERTS];
-    __shared__ float wv[kRouteThreads / 32];
-    __shared__ int wi[kRouteThreads / 32];
-    __shared__ int sel[HFQ_MAX_TOPK];
-    const int t = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const float *l = logits + (size_t)t * E;
-    for (int e = tid; e < E; e += blockDim.x) {
-        sl[e] = l[e];
-        taken[e] = 0;
-    }
-    __syncthreads();
-    for (int j = 0; j < k; ++j) {
-        float bv = -INFINITY;
-        int bi = 0x7fffffff;
-        for (int e = tid; e < E; e += blockDim.x)
-            if (!taken[e] && better(sl[e], e, bv, bi)) { bv = sl[e]; bi = e; }
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-            float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-            int oi = __shfl_xor_sync(0xffffffffu, bi, o);
-            if (better(ov, oi, bv, bi)) { bv = ov; bi = oi; }
-        }
-        if (lane == 0) { wv[warp] = bv; wi[warp] = bi; }
-        __syncthreads();
-        if (tid == 0) {
-            float b = wv[0];
-            int ib = wi[0];
-            for (int w = 1; w < (int)(blockDim.x / 32); ++w)
-                if (better(wv[w], wi[w], b, ib)) { b = wv[w]; ib = wi[w]; }
-            sel[j] = ib;
-            taken[ib] = 1;
-        }
-        __syncthreads();
-    }
-    if (tid == 0) {
-        // renormalised weights = softmax over the selected logits; slot 0 is the max
-        float m = sl[sel[0]], s = 0.0f, ex[HFQ_MAX_TOPK];
-        for (int j = 0; j < k; ++j) { ex[j] = __expf(sl[sel[j]] - m); s += ex[j]; }
-        for (int j = 0; j < k; ++j) {
-            idx[(size_t)t * k + j] = sel[j];
-            wts[(size_t)t * k + j] = ex[j] / s;
-        }
+    const int t = blockIdx.x * kRouteWarps + (threadIdx.x >> 5), lane = threadIdx.x & 31;
+    if (t >= T) return;                         // whole warps
+    int e;
+    float w;
+    warp_route(logits + (size_t)t * E, E, k, e, w);
+    if (lane < k) {
+        idx[(size_t)t * k + lane] = e;
+        wts[(size_t)t * k + lane] = w;
     }
 }
 
 // Grouping by expert, stable: three passes over chunks of kGroupChunk pairs.
-constexpr int kGroupChunk = 256;
+constexpr int kGroupChunk = 512;
 
 __global__ void group_hist_kernel(const int32_t *__restrict__ idx, int P, int E,
                                   int32_t *__restrict__ hist)
@@ -180,9 +142,16 @@ __global__ void group_scan_kernel(int32_t *__restrict__ hist, int n_chunks, int 
                                   int32_t *__restrict__ cnt, int32_t *__restrict__ off)
 {
     __shared__ int tot[HFQ_MAX_EXPERTS + 1];
+    constexpr int kU = 16;                      // chunk counts in flight per thread
     for (int e = threadIdx.x; e < E; e += blockDim.x) {
         int s = 0;
-        for (int c = 0; c < n_chunks; ++c) s += hist[(size_t)c * E + e];
+        for (int c0 = 0; c0 < n_chunks; c0 += kU) {
+            int v[kU];
+#pragma unroll
+            for (int u = 0; u < kU; ++u) v[u] = c0 + u < n_chunks ? hist[(size_t)(c0 + u) * E + e] : 0;
+#pragma unroll
+            for (int u = 0; u < kU; ++u) s += v[u];
+        }
         tot[e] = s;
         cnt[e] = s;
     }
@@ -196,10 +165,16 @@ __global__ void group_scan_kernel(int32_t *__restrict__ hist, int n_chunks, int 
     __syncthreads();
     for (int e = threadIdx.x; e < E; e += blockDim.x) {
         int base = tot[e];
-        for (int c = 0; c < n_chunks; ++c) {
-            int v = hist[(size_t)c * E + e];
-            hist[(size_t)c * E + e] = base;
-            base += v;
+        for (int c0 = 0; c0 < n_chunks; c0 += kU) {
+            int v[kU];
+#pragma unroll
+            for (int u = 0; u < kU; ++u) v[u] = c0 + u < n_chunks ? hist[(size_t)(c0 + u) * E + e] : 0;
+#pragma unroll
+            for (int u = 0; u < kU; ++u)
+                if (c0 + u < n_chunks) {
+                    hist[(size_t)(c0 + u) * E + e] = base;
+                    base += v[u];
+                }
         }
     }
 }
@@ -315,7 +290,7 @@ hfq_status moe_route(const float *logits, int T, int E, int k, int32_t *idx, flo
     if (group && (!workspace || ws_bytes < need))
         return fail(HFQ_ERR_WORKSPACE, "moe_route: grouping needs %zu bytes of workspace", need);
     cudaStream_t s = (cudaStream_t)stream;
-    route_kernel<<<T, kRouteThreads, 0, s>>>(logits, E, k, idx, wts);
+    route_kernel<<<(T + kRouteWarps - 1) / kRouteWarps, kRouteWarps * 32, 0, s>>>(logits, T, E, k, idx, wts);
     if (group) {
         int P = T * k;
         int chunks = (P + kGroupChunk - 1) / kGroupChunk;

@@ -21,9 +21,9 @@ namespace {
 constexpr int kM = 128;                    // weight rows per tile (MMA M)
 constexpr int kN = 128;                    // token pairs per tile (MMA N)
 constexpr int kKC = 128;                   // K per pipeline stage (8 MMAs of K = 16)
-constexpr int kWGU = kKC / 16;             // 8-byte nibble words per row and chunk (gate/up)
-constexpr int kWD = kKC / 32;              // per half row (down: two threads per row)
-constexpr int kTcThr = 256;                // 8 warps
+constexpr int kQB = kKC / 32;              // 16-byte nibble quarters per row and chunk (4)
+constexpr int kTcThr = 512;                // 16 warps
+constexpr int kTcW = kTcThr / 32;
 constexpr int kTileBytes = kM * kKC * 2;   // one 128 x kKC bf16 operand tile
 constexpr uint32_t kLbo = (kM / 8) * 128;  // bytes between 8-element K chunks (2048)
 constexpr uint32_t kSbo = 128;             // bytes between 8-row groups
@@ -48,26 +48,44 @@ __device__ __forceinline__ uint32_t tile_off(int row, int k8)
     return (uint32_t)(row >> 3) * kSbo + (uint32_t)(row & 7) * 16u + (uint32_t)k8 * kLbo;
 }
 
+// Two f32 in one 64-bit register (low word first) and back.
+__device__ __forceinline__ unsigned long long f32x2(float lo, float hi)
+{
+    unsigned long long r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+
+__device__ __forceinline__ unsigned long long u32x2(uint32_t lo, uint32_t hi)
+{
+    unsigned long long r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "r"(lo), "r"(hi));
+    return r;
+}
+
 // 8 nibbles -> 8 bf16 weights RN_bf16(fmaf(scale, q, zero)), elements in order.
+// The packed two-wide f32 add and FMA of sm_100 round each lane like their
+// scalar forms, so the weights are the same bits as with scalar fmaf.
 __device__ __forceinline__ uint4 deq8(uint32_t w, float scale, float zero)
 {
     const uint32_t lo = w & 0x0F0F0F0Fu, hi = (w >> 4) & 0x0F0F0F0Fu;
-    float f[8];
+    const unsigned long long off = f32x2(-8388608.0f, -8388608.0f);
+    const unsigned long long sc = f32x2(scale, scale), ze = f32x2(zero, zero);
+    uint32_t r[4];
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
         // 0x4B0000qq = 2^23 + q exactly; subtracting 2^23 is exact
-        const float qe = __uint_as_float(__byte_perm(lo, 0x4B000000u, 0x7440u | j)) - 8388608.0f;
-        const float qo = __uint_as_float(__byte_perm(hi, 0x4B000000u, 0x7440u | j)) - 8388608.0f;
-        f[2 * j] = fmaf(scale, qe, zero);
-        f[2 * j + 1] = fmaf(scale, qo, zero);
+        const uint32_t qe = __byte_perm(lo, 0x4B000000u, 0x7440u | j);
+        const uint32_t qo = __byte_perm(hi, 0x4B000000u, 0x7440u | j);
+        unsigned long long q2;
+        asm("add.rn.f32x2 %0, %1, %2;" : "=l"(q2) : "l"(u32x2(qe, qo)), "l"(off));
+        asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(q2) : "l"(sc), "l"(q2), "l"(ze));
+        float fe, fo;
+        asm("mov.b64 {%0, %1}, %2;" : "=f"(fe), "=f"(fo) : "l"(q2));
+        const __nv_bfloat162 b = __floats2bfloat162_rn(fe, fo);
+        r[j] = *reinterpret_cast<const uint32_t *>(&b);
     }
-    uint4 r;
-    __nv_bfloat162 b;
-    b = __floats2bfloat162_rn(f[0], f[1]); r.x = *reinterpret_cast<uint32_t *>(&b);
-    b = __floats2bfloat162_rn(f[2], f[3]); r.y = *reinterpret_cast<uint32_t *>(&b);
-    b = __floats2bfloat162_rn(f[4], f[5]); r.z = *reinterpret_cast<uint32_t *>(&b);
-    b = __floats2bfloat162_rn(f[6], f[7]); r.w = *reinterpret_cast<uint32_t *>(&b);
-    return r;
+    return make_uint4(r[0], r[1], r[2], r[3]);
 }
 
 __device__ bool tc_wait(const TcArgs &a, uint64_t *bar, uint32_t parity, int &abort)
@@ -119,14 +137,20 @@ __global__ void __launch_bounds__(kTcThr, 1) tc_kernel(const __grid_constant__ T
     uint32_t chunk = 0;                              // stages used so far (buffer = chunk & 1)
     const int total = a.item_off[a.E];
 
-    // this thread's weight row (gate/up: one matrix; down: half of each K
-    // chunk) and activation pieces; the next chunk's loads (of this item or,
-    // at its last chunk, of the next item) are in flight while a chunk is
-    // dequantised and multiplied
-    const int row = tid & (kM - 1), which = tid >> 7;
+    // Loads: a warp instruction reads 8 rows x 64 contiguous bytes (4 lanes
+    // of 16 bytes per row, rows fastest across lanes), and the 8 lanes of each
+    // shared-memory store phase write one 128-byte core-matrix column (8
+    // consecutive rows, one K chunk).  Weight rows: rid = (lane & 7) +
+    // 8 * (warp + kTcW * i), i < kRI (gate/up: rows >= 128 are the up
+    // matrix), quarter qq = lane >> 3.  Activation pieces: token n =
+    // (lane & 7) + 8 * (b & 15), K piece 4 * (b >> 4) + qq, b = warp + kTcW * i.
+    // The next chunk's loads (of this item or, at its last chunk, of the next
+    // item) are in flight while a chunk is dequantised and multiplied.
+    constexpr int kRI = (GU ? 2 * kM : kM) / (8 * kTcW);   // weight rows per thread and chunk
+    const int qq = lane >> 3, rl = lane & 7;
     struct Geo {
         int p0, nvalid, r0;
-        const uint8_t *rrow;
+        const uint8_t *gbase, *ubase;                // gate (or down) and up matrices
     };
     auto geo_of = [&](int item) {
         int lo = 0, hi = a.E;                        // item_off[lo] <= item < item_off[lo + 1]
@@ -141,25 +165,30 @@ __global__ void __launch_bounds__(kTcThr, 1) tc_kernel(const __grid_constant__ T
         g.nvalid = min(kN, a.cnt[e] - nt * kN);
         g.r0 = rt * kM;
         const uint8_t *base = static_cast<const uint8_t *>(a.eptr[e]);
-        const uint8_t *A = GU ? (which ? base + mg : base) : base + 2 * mg;   // gate / up, or down
-        g.rrow = A + (size_t)(g.r0 + row) * rowB;
+        g.gbase = (GU ? base : base + 2 * mg) + (size_t)g.r0 * rowB;
+        g.ubase = base + mg + (size_t)g.r0 * rowB;
         return g;
     };
-    float2 nsz;
-    uint2 nw[kWGU];
+    float2 nsz[kRI];
+    uint4 nw[kRI];
     uint4 nx[(kN * kKC / 8) / kTcThr];
     auto load = [&](const Geo &g, int kc2) {
         const int blk = (kc2 * kKC) / kBlock, sub = ((kc2 * kKC) % kBlock) / 2;   // nibble byte
-        const uint8_t *rp = g.rrow + (size_t)blk * kBlockBytes;
-        nsz = __ldg(reinterpret_cast<const float2 *>(rp));
 #pragma unroll
-        for (int i = 0; i < kWGU; ++i)
-            if (GU || i < kWD)
-                nw[i] = __ldg(reinterpret_cast<const uint2 *>(rp + 8 + sub + (GU ? 0 : 8 * kWD * which) + 8 * i));
+        for (int i = 0; i < kRI; ++i) {
+            const int rid = rl + 8 * (warp + kTcW * i);
+            const uint8_t *rp = (GU && rid >= kM ? g.ubase : g.gbase) + (size_t)(rid & (kM - 1)) * rowB +
+                                (size_t)blk * kBlockBytes;
+            nsz[i] = __ldg(reinterpret_cast<const float2 *>(rp));
+            // the payload of an even block starts at 8 mod 16: two 8-byte loads
+            const uint2 lo = __ldg(reinterpret_cast<const uint2 *>(rp + 8 + sub + 16 * qq));
+            const uint2 hi = __ldg(reinterpret_cast<const uint2 *>(rp + 16 + sub + 16 * qq));
+            nw[i] = make_uint4(lo.x, lo.y, hi.x, hi.y);
+        }
 #pragma unroll
         for (int i = 0; i < (kN * kKC / 8) / kTcThr; ++i) {
-            const int id = tid + i * kTcThr;
-            const int n = id & (kN - 1), k8 = id >> 7;
+            const int blkid = warp + kTcW * i;
+            const int n = rl + 8 * (blkid & 15), k8 = 4 * (blkid >> 4) + qq;
             nx[i] = n < g.nvalid ? __ldg(reinterpret_cast<const uint4 *>(a.xin + (size_t)(g.p0 + n) * K + kc2 * kKC + k8 * 8))
                                  : make_uint4(0u, 0u, 0u, 0u);
         }
@@ -179,11 +208,11 @@ __global__ void __launch_bounds__(kTcThr, 1) tc_kernel(const __grid_constant__ T
         for (int kc = 0; kc < nK; ++kc, ++chunk) {
             const int s = chunk & 1;
             uint8_t *st = smem + (size_t)s * kOps * kTileBytes;
-            const float2 sz = nsz;
-            uint2 w[kWGU];
+            float2 sz[kRI];
+            uint4 w[kRI];
             uint4 xv[(kN * kKC / 8) / kTcThr];
 #pragma unroll
-            for (int i = 0; i < kWGU; ++i) w[i] = nw[i];
+            for (int i = 0; i < kRI; ++i) { sz[i] = nsz[i]; w[i] = nw[i]; }
 #pragma unroll
             for (int i = 0; i < (kN * kKC / 8) / kTcThr; ++i) xv[i] = nx[i];
             if (!abort) {
@@ -192,26 +221,23 @@ __global__ void __launch_bounds__(kTcThr, 1) tc_kernel(const __grid_constant__ T
             }
             if (commits[s] && !abort) tc_wait(a, &mma_bar[s], (commits[s] - 1) & 1, abort);
             if (!abort) {
-                uint8_t *dst = st + (GU && which ? kTileBytes : 0);
-                if (GU) {
+                // weights: row rid, K pieces 4 qq .. 4 qq + 3 of this chunk
 #pragma unroll
-                    for (int i = 0; i < kWGU; ++i) {
-                        *reinterpret_cast<uint4 *>(dst + tile_off(row, 2 * i)) = deq8(w[i].x, sz.x, sz.y);
-                        *reinterpret_cast<uint4 *>(dst + tile_off(row, 2 * i + 1)) = deq8(w[i].y, sz.x, sz.y);
-                    }
-                } else {
-#pragma unroll
-                    for (int i = 0; i < kWD; ++i) {
-                        *reinterpret_cast<uint4 *>(dst + tile_off(row, 2 * kWD * which + 2 * i)) = deq8(w[i].x, sz.x, sz.y);
-                        *reinterpret_cast<uint4 *>(dst + tile_off(row, 2 * kWD * which + 2 * i + 1)) = deq8(w[i].y, sz.x, sz.y);
-                    }
+                for (int i = 0; i < kRI; ++i) {
+                    const int rid = rl + 8 * (warp + kTcW * i);
+                    uint8_t *dst = st + (GU && rid >= kM ? kTileBytes : 0);
+                    const int rr = rid & (kM - 1);
+                    *reinterpret_cast<uint4 *>(dst + tile_off(rr, 4 * qq + 0)) = deq8(w[i].x, sz[i].x, sz[i].y);
+                    *reinterpret_cast<uint4 *>(dst + tile_off(rr, 4 * qq + 1)) = deq8(w[i].y, sz[i].x, sz[i].y);
+                    *reinterpret_cast<uint4 *>(dst + tile_off(rr, 4 * qq + 2)) = deq8(w[i].z, sz[i].x, sz[i].y);
+                    *reinterpret_cast<uint4 *>(dst + tile_off(rr, 4 * qq + 3)) = deq8(w[i].w, sz[i].x, sz[i].y);
                 }
-                // activations: 128 token rows x 64 values, 16 bytes per piece
+                // activations: 128 token rows x kKC values, 16 bytes per piece
                 uint8_t *bt = st + (size_t)(kOps - 1) * kTileBytes;
 #pragma unroll
                 for (int i = 0; i < (kN * kKC / 8) / kTcThr; ++i) {
-                    const int id = tid + i * kTcThr;
-                    const int n = id & (kN - 1), k8 = id >> 7;
+                    const int blkid = warp + kTcW * i;
+                    const int n = rl + 8 * (blkid & 15), k8 = 4 * (blkid >> 4) + qq;
                     *reinterpret_cast<uint4 *>(bt + tile_off(n, k8)) = xv[i];
                 }
             }
@@ -239,11 +265,12 @@ __global__ void __launch_bounds__(kTcThr, 1) tc_kernel(const __grid_constant__ T
         if (!abort && !s_abort) tc_wait(a, &mma_bar[sl], (commits[sl] - 1) & 1, abort);
         tc_fence_after_sync();
         if (!abort && !s_abort) {
-            const int lg = warp & 3, half = warp >> 2;          // TMEM lane group, column half
+            constexpr int kCols = kN / (kTcW / 4);                // columns per warp
+            const int lg = warp & 3, half = warp >> 2;          // TMEM lane group, column group
             const int r = lg * 32 + lane;
             const uint32_t trow = tmem + ((uint32_t)(lg * 32) << 16);
 #pragma unroll 1
-            for (int c = half * (kN / 2); c < (half + 1) * (kN / 2); c += 16) {
+            for (int c = half * kCols; c < (half + 1) * kCols; c += 16) {
                 float g[16], u[16];
                 tmem_ld16(trow + c, g);
                 if (GU) tmem_ld16(trow + kN + c, u);
