@@ -33,7 +33,8 @@ struct TcArgs {
     const void *const *eptr;       // [E] expert base addresses
     const int32_t *cnt, *off, *perm;
     const float *wts;              // [T*k] routing weights, flat
-    const uint16_t *xin;           // gate/up: X_perm [T*k][H]; down: H_perm [T*k][I] (bf16)
+    const uint16_t *xin;           // gate/up: X_perm [T*k][H] or x [T][H]; down: H_perm [T*k][I] (bf16)
+    int x_direct;                  // gate/up reads row perm[q] / k of x instead of row q of X_perm
     uint16_t *hout;                // gate/up: H_perm out
     float *o;                      // down: O [T*k][H] f32, row q = pair perm[q]
     const int32_t *item_off;       // [E+1] prefix of work items of this phase
@@ -151,7 +152,10 @@ __global__ void __launch_bounds__(kTcThr, 1) tc_kernel(const __grid_constant__ T
     struct Geo {
         int p0, nvalid, r0;
         const uint8_t *gbase, *ubase;                // gate (or down) and up matrices
+        const uint16_t *xrow;                        // this thread's activation row, or null
     };
+    static_assert(kTcW == 16, "one activation row per thread: n = (lane & 7) + 8 * warp");
+    const int xn = rl + 8 * warp;
     auto geo_of = [&](int item) {
         int lo = 0, hi = a.E;                        // item_off[lo] <= item < item_off[lo + 1]
         while (hi - lo > 1) {
@@ -167,6 +171,11 @@ __global__ void __launch_bounds__(kTcThr, 1) tc_kernel(const __grid_constant__ T
         const uint8_t *base = static_cast<const uint8_t *>(a.eptr[e]);
         g.gbase = (GU ? base : base + 2 * mg) + (size_t)g.r0 * rowB;
         g.ubase = base + mg + (size_t)g.r0 * rowB;
+        g.xrow = nullptr;
+        if (xn < g.nvalid) {
+            const int q = g.p0 + xn;
+            g.xrow = a.xin + (size_t)(GU && a.x_direct ? a.perm[q] / a.k : q) * K;
+        }
         return g;
     };
     float2 nsz[kRI];
@@ -187,10 +196,9 @@ __global__ void __launch_bounds__(kTcThr, 1) tc_kernel(const __grid_constant__ T
         }
 #pragma unroll
         for (int i = 0; i < (kN * kKC / 8) / kTcThr; ++i) {
-            const int blkid = warp + kTcW * i;
-            const int n = rl + 8 * (blkid & 15), k8 = 4 * (blkid >> 4) + qq;
-            nx[i] = n < g.nvalid ? __ldg(reinterpret_cast<const uint4 *>(a.xin + (size_t)(g.p0 + n) * K + kc2 * kKC + k8 * 8))
-                                 : make_uint4(0u, 0u, 0u, 0u);
+            const int k8 = 4 * ((warp + kTcW * i) >> 4) + qq;
+            nx[i] = g.xrow ? __ldg(reinterpret_cast<const uint4 *>(g.xrow + kc2 * kKC + k8 * 8))
+                           : make_uint4(0u, 0u, 0u, 0u);
         }
     };
     Geo cur{};
@@ -327,6 +335,13 @@ __global__ void tc_plan_kernel(const int32_t *__restrict__ cnt, int E, int I, in
     }
 }
 
+// pos[perm[q]] = q (the gate/up kernel reads bf16 x through perm itself).
+__global__ void tc_pos_kernel(const int32_t *__restrict__ perm, int P, int32_t *__restrict__ pos)
+{
+    for (int q = blockIdx.x * blockDim.x + threadIdx.x; q < P; q += gridDim.x * blockDim.x)
+        pos[perm[q]] = q;
+}
+
 // X_perm[q] = x[token of pair perm[q]] as bf16 (16 bytes per thread step);
 // pos[perm[q]] = q.
 __global__ void tc_gather_kernel(const void *__restrict__ x, int x_f32, const int32_t *__restrict__ perm,
@@ -437,14 +452,19 @@ hfq_status launch_tc(const hfq4_layer &L, const void *x, bool x_f32, int T, int 
     }
     tc_plan_kernel<<<1, 512, 0, s>>>(cnt, E, I, H, gu_off, dn_off);
     const size_t n8 = P * H / 8;
-    tc_gather_kernel<<<(unsigned)std::min<size_t>((n8 + 255) / 256, (size_t)tc_sms() * 16), 256, 0, s>>>(
-        x, x_f32 ? 1 : 0, perm, (int)P, k, H, xp, pos);
+    if (x_f32)
+        tc_gather_kernel<<<(unsigned)std::min<size_t>((n8 + 255) / 256, (size_t)tc_sms() * 16), 256, 0, s>>>(
+            x, 1, perm, (int)P, k, H, xp, pos);
+    else
+        tc_pos_kernel<<<(unsigned)std::min<size_t>((P + 255) / 256, (size_t)tc_sms() * 4), 256, 0, s>>>(
+            perm, (int)P, pos);
     TcArgs a;
     a.eptr = L.expert_ptr; a.cnt = cnt; a.off = off; a.perm = perm; a.wts = wts;
     a.status = status; a.timeout_ns = timeout_ns; a.E = E; a.H = H; a.I = I; a.k = k;
-    a.xin = xp; a.hout = hp; a.o = nullptr; a.item_off = gu_off;
+    a.xin = x_f32 ? xp : static_cast<const uint16_t *>(x); a.x_direct = x_f32 ? 0 : 1;
+    a.hout = hp; a.o = nullptr; a.item_off = gu_off;
     tc_kernel<true><<<tc_sms(), kTcThr, smem_gu, s>>>(a);
-    a.xin = hp; a.hout = nullptr; a.o = ob; a.item_off = dn_off;
+    a.xin = hp; a.x_direct = 0; a.hout = nullptr; a.o = ob; a.item_off = dn_off;
     tc_kernel<false><<<tc_sms(), kTcThr, smem_dn, s>>>(a);
     const size_t n4 = (size_t)T * H / 4;
     tc_combine_kernel<<<(unsigned)std::min<size_t>((n4 + 255) / 256, (size_t)tc_sms() * 16), 256, 0, s>>>(
