@@ -197,6 +197,24 @@ def measure_hbm_read(torch, eo, nbytes=4 << 30):
     return round(3 * nbytes / (e0.elapsed_time(e1) / 1e3) / 1e9, 1)
 
 
+def max_over_ranks(dist, values, device):
+    """Each value's maximum over all ranks (a replicated job takes as long as
+    its slowest rank); the values unchanged without a process group."""
+    if dist is None:
+        return [float(v) for v in values]
+    import torch
+
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(v) for v in t]
+
+
+def job_rate(world, steps, units_per_step, job_ms):
+    """Whole-job throughput: the units all `world` replicas processed in
+    `steps` steps, over the job's time."""
+    return world * steps * units_per_step / (job_ms / 1e3)
+
+
 def run_ours(args, rank, world, local_rank):
     import numpy as np
     import torch
@@ -322,15 +340,12 @@ def run_ours(args, rank, world, local_rank):
     e2e_ms = e0.elapsed_time(e1)
     eo.hfq_workspace_status(ws, stream)
 
-    if dist:
-        t = torch.tensor([total_ms, e2e_ms], dtype=torch.float64, device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms, e2e_ms = float(t[0]), float(t[1])
+    total_ms, e2e_ms = max_over_ranks(dist, [total_ms, e2e_ms], "cuda")
 
     hbm_b = sum(per_group[i % G][0] for i in range(K)) / K
     host_b = sum(per_group[i % G][1] for i in range(K)) / K
     bytes_per_step = hbm_b + host_b
-    value = world * K * T / (total_ms / 1e3)
+    value = job_rate(world, K, T, total_ms)
     mean_launch_ms = sum(per_launch) / K
     peak, peak_kind = peaks()
     out = {
@@ -391,7 +406,7 @@ def run_ours(args, rank, world, local_rank):
                            "mean_launch_ms": round(mean_launch_ms, 5)}
         if args.hbm_read_probe:
             out["roofline"]["hbm_read_probe_gbs"] = measure_hbm_read(torch, eo)
-    out["e2e"] = {"value": round(world * K2 * T / (e2e_ms / 1e3), 2), "unit": "tokens/s",
+    out["e2e"] = {"value": round(job_rate(world, K2, T, e2e_ms), 2), "unit": "tokens/s",
                   "h2d_bytes_per_step": int(in_l.numel() * 4 + in_x.numel() * 2),
                   "d2h_bytes_per_step": int(out_x.numel() * 2)}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
