@@ -251,10 +251,12 @@ __global__ void __launch_bounds__(kThr, 1) decode1_kernel(const __grid_constant_
                 __syncwarp();
                 stamp_dep(a, l, 26, lane == 0, 0.f);
                 if (lane < k && !loc) {
+                    // expert bytes are read once per step: evict them first from L2
+                    const uint64_t pol = l2_evict_first_policy();
                     uint8_t *slot = slots + (size_t)lane * a.slot_bytes;
-                    if (sg.len) bulk_g2s(slot, base + sg.src, (uint32_t)sg.len, &sh.gu_bar[lane]);
-                    if (su.len) bulk_g2s(slot + a.up_off, base + su.src, (uint32_t)su.len, &sh.gu_bar[lane]);
-                    if (sd.len) bulk_g2s(slot + a.down_off, base + sd.src, (uint32_t)sd.len, &sh.d_bar[lane]);
+                    if (sg.len) bulk_g2s_hint(slot, base + sg.src, (uint32_t)sg.len, &sh.gu_bar[lane], pol);
+                    if (su.len) bulk_g2s_hint(slot + a.up_off, base + su.src, (uint32_t)su.len, &sh.gu_bar[lane], pol);
+                    if (sd.len) bulk_g2s_hint(slot + a.down_off, base + sd.src, (uint32_t)sd.len, &sh.d_bar[lane], pol);
                 }
                 if (lane == 0) { sh.armed = l + 1; sh.hostmask = hm; }
                 __syncwarp();

@@ -363,13 +363,15 @@ __global__ void __launch_bounds__(kThr, 1) verify_kernel(const __grid_constant__
                 if (lane == 0) sh.armed_seq[s] = seq;
                 if (!sh.uloc[u]) {
                     if (lane == 0) {
+                        // expert bytes are read once per step: evict them first from L2
+                        const uint64_t pol = l2_evict_first_policy();
                         if (i < U) {
                             mbar_arrive_expect_tx(&sh.full[s], (uint32_t)(sg.len + su.len));
-                            if (sg.len) bulk_g2s(st, base + sg.src, (uint32_t)sg.len, &sh.full[s]);
-                            if (su.len) bulk_g2s(st + up_off, base + su.src, (uint32_t)su.len, &sh.full[s]);
+                            if (sg.len) bulk_g2s_hint(st, base + sg.src, (uint32_t)sg.len, &sh.full[s], pol);
+                            if (su.len) bulk_g2s_hint(st + up_off, base + su.src, (uint32_t)su.len, &sh.full[s], pol);
                         } else {
                             mbar_arrive_expect_tx(&sh.full[s], (uint32_t)sd.len);
-                            if (sd.len) bulk_g2s(st, base + sd.src, (uint32_t)sd.len, &sh.full[s]);
+                            if (sd.len) bulk_g2s_hint(st, base + sd.src, (uint32_t)sd.len, &sh.full[s], pol);
                         }
                     }
                 } else {
