@@ -154,6 +154,24 @@ def test_route_ties_and_degenerate_cases(eo):
     _check_route(eo, np.random.default_rng(3).standard_normal((2, 1)).astype(np.float32), 1)
 
 
+def test_route_winners_concentrated_in_one_lane(eo):
+    """All selected experts among one lane's contiguous keys of the warp
+    top-k (experts 8 i .. 8 i + 7 at E = 256, 16 i .. at E = 512): the lane
+    wins every round and refills its cached top three after each third win."""
+    rng = np.random.default_rng(5)
+    l = rng.standard_normal((6, 256)).astype(np.float32)
+    l[0, 0:8] += 10.0                           # lane 0 holds the top 8
+    l[1, 248:256] += 10.0                       # the last lane
+    l[2, 40:48] = 9.0                           # eight equal winners in one lane
+    l[3, 40:44] += 10.0                         # four from one lane, four from others
+    l[3, [3, 77, 130, 201]] += 9.0
+    _check_route(eo, l, 8)
+    l2 = rng.standard_normal((3, 512)).astype(np.float32)
+    l2[0, 16:32] += 10.0                        # one lane's 16 keys are the top 16
+    l2[1, 496:512] = 5.0
+    _check_route(eo, l2, 16)
+
+
 # ---------------------------------------------------------------- forward
 
 def test_forward_tiny_workload_all_tokens(eo):
