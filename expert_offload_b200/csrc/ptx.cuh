@@ -42,6 +42,15 @@ __device__ __forceinline__ void mbar_arrive(uint64_t *bar)
                  : "memory");
 }
 
+// `count` arrivals on `bar` at once.
+__device__ __forceinline__ void mbar_arrive_cnt(uint64_t *bar, uint32_t count)
+{
+    asm volatile("{ .reg .b64 st; mbarrier.arrive.release.cta.shared::cta.b64 st, [%0], %1; }" ::"r"(
+                     smem_u32(bar)),
+                 "r"(count)
+                 : "memory");
+}
+
 // Arrives once on `bar` and raises its expected transaction bytes by `bytes`.
 __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t bytes)
 {

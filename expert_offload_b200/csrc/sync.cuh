@@ -45,6 +45,23 @@ __device__ inline bool wait_counter_ge(const WaitCtx &w, const unsigned *p, unsi
     }
 }
 
+// Waits until the producer has armed use `seq` of a ring stage (*armed ==
+// seq), so that a following parity wait on the stage's full barrier cannot
+// match an earlier use of the same parity.
+__device__ inline bool wait_armed(const WaitCtx &w, const int *armed, int seq)
+{
+    uint64_t t0 = 0;
+    for (int it = 0;; ++it) {
+        if (*(const volatile int *)armed == seq) return true;
+        if (*w.abort) return false;
+        if (it == 64) t0 = globaltimer_ns();
+        if (it > 64 && (it & 15) == 0 && deadline_passed(t0, w.timeout_ns)) {
+            raise_timeout(w);
+            return false;
+        }
+    }
+}
+
 // Waits for the phase of `bar` with the given parity to complete.
 __device__ inline bool wait_mbar_phase(const WaitCtx &w, uint64_t *bar, uint32_t parity)
 {

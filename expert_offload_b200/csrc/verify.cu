@@ -360,7 +360,14 @@ __global__ void __launch_bounds__(kThr, 1) verify_kernel(const __grid_constant__
                     break;
                 }
                 uint8_t *st = ring + (size_t)s * a.stage_bytes;
-                if (lane == 0) sh.armed_seq[s] = seq;
+                if (lane == 0) {
+                    sh.armed_seq[s] = seq;
+                    // consumer warps with no pair in this item do not touch the
+                    // stage: release it for them in this use's phase (pairs of an
+                    // item are contiguous and go to warps p mod kCW)
+                    const int np = min(kCW, sh.pair0[u + 1] - sh.pair0[u]);
+                    if (np < kCW) mbar_arrive_cnt(&sh.empty[s], (uint32_t)(kCW - np));
+                }
                 if (!sh.uloc[u]) {
                     if (lane == 0) {
                         // expert bytes are read once per step: evict them first from L2
@@ -405,19 +412,22 @@ __global__ void __launch_bounds__(kThr, 1) verify_kernel(const __grid_constant__
             for (int u = 0; u < U; ++u) {
                 const int seq = stage_base + u, s = seq % NS;
                 const uint8_t *st = ring + (size_t)s * a.stage_bytes;
-                // every warp waits for the item before it releases the stage, with
-                // or without pairs in it: an arrival on the empty barrier of a use
-                // that is not armed yet would count toward the previous use
+                int p = sh.pair0[u] + ((warp - sh.pair0[u]) % kCW + kCW) % kCW;
+                // items without a pair of this warp are skipped: the producer
+                // released the stage for this warp when it armed the item
+                if (p >= sh.pair0[u + 1]) continue;
                 if (ok) {
                     int w = 1;
                     if (lane == 0) {
-                        w = wait_mbar_phase(wc, &sh.full[s], (seq / NS) & 1) ? 1 : 0;
+                        // this use armed first: the full barrier's earlier uses
+                        // are then complete and the parity names this use alone
+                        w = (wait_armed(wc, &sh.armed_seq[s], seq) &&
+                             wait_mbar_phase(wc, &sh.full[s], (seq / NS) & 1)) ? 1 : 0;
                         note_wait(a, w, 2, l, seq);
                     }
                     ok = __shfl_sync(0xffffffffu, w, 0) != 0;
                     vstamp(a, l, 3, lane == 0 && u == 0 && warp == 0);
                 }
-                int p = sh.pair0[u] + ((warp - sh.pair0[u]) % kCW + kCW) % kCW;
                 for (; p < sh.pair0[u + 1] && ok; p += kCW) {
                     uint32_t X[32];
                     int xe = 0;
@@ -521,17 +531,8 @@ __global__ void __launch_bounds__(kThr, 1) verify_kernel(const __grid_constant__
                 const int seq = stage_base + U + u, s = seq % NS;
                 const uint8_t *st = ring + (size_t)s * a.stage_bytes;
                 bool waited = false;
-                if (ok && pnext >= sh.pair0[u + 1]) {
-                    // no pair of this warp in the item: still wait for it before
-                    // releasing the stage (see the gate/up loop)
-                    int w = 1;
-                    if (lane == 0) {
-                        w = wait_mbar_phase(wc, &sh.full[s], (seq / NS) & 1) ? 1 : 0;
-                        note_wait(a, w, 4, l, seq);
-                    }
-                    ok = __shfl_sync(0xffffffffu, w, 0) != 0;
-                    waited = true;
-                }
+                // no pair of this warp in the item: skipped (released by the producer)
+                if (pnext >= sh.pair0[u + 1]) continue;
                 while (ok && pnext < sh.pair0[u + 1]) {
                     const int p = pnext;
                     float *hw = hw0 + (size_t)buf * Pl * kHStride;
@@ -557,7 +558,8 @@ __global__ void __launch_bounds__(kThr, 1) verify_kernel(const __grid_constant__
                     if (!waited) {
                         int w = 1;
                         if (lane == 0) {
-                            w = wait_mbar_phase(wc, &sh.full[s], (seq / NS) & 1) ? 1 : 0;
+                            w = (wait_armed(wc, &sh.armed_seq[s], seq) &&
+                                 wait_mbar_phase(wc, &sh.full[s], (seq / NS) & 1)) ? 1 : 0;
                             note_wait(a, w, 4, l, seq);
                         }
                         ok = __shfl_sync(0xffffffffu, w, 0) != 0;
