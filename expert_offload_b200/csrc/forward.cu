@@ -285,12 +285,15 @@ hfq_status hfq4_moe_forward(const hfq4_layer *layer, const void *x, hfq_dtype x_
     char *wsb = static_cast<char *>(workspace);
     float *h = reinterpret_cast<float *>(wsb + stack_ctl_bytes());
     cudaStream_t s = (cudaStream_t)stream;
-    const bool use_tc = path == HFQ_PATH_TC || (path == HFQ_PATH_AUTO && T > 8 && grouped);
+    const bool use_tc = path == HFQ_PATH_TC ||
+                        (path == HFQ_PATH_AUTO && T > 8 && grouped && tc_supported(layer->hidden, layer->inter));
     if (use_tc) {
         if (!grouped)
             return fail(HFQ_ERR_ARG, "the tensor-core path needs cnt, off and perm from moe_route");
         if (!tc_supported(layer->hidden, layer->inter))
-            return fail(HFQ_ERR_UNSUPPORTED, "tensor-core path: hidden and inter must be multiples of 128");
+            return fail(HFQ_ERR_UNSUPPORTED,
+                        "tensor-core path: hidden and inter must be multiples of 128 with an even number of "
+                        "256-weight blocks per row (hidden %d, inter %d)", layer->hidden, layer->inter);
         st = launch_tc(*layer, x, x_dtype == HFQ_F32, T, k, cnt, off, perm, wts, y,
                        static_cast<uint16_t *>(y_bf16), wsb + stack_ctl_bytes() + h_bytes(T, k, layer->inter),
                        static_cast<unsigned *>(workspace), option_wait_timeout_ns(), s);

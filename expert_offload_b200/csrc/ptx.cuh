@@ -111,6 +111,63 @@ __device__ __forceinline__ void cp_async16(void *dst, const void *src)
                  : "memory");
 }
 
+// 8-byte asynchronous copy global -> shared (both 8-byte aligned; cached in L1).
+__device__ __forceinline__ void cp_async8(void *dst, const void *src)
+{
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(smem_u32(dst)), "l"(src)
+                 : "memory");
+}
+
+// Waits until at most N committed groups of this thread are still in flight.
+template <int N>
+__device__ __forceinline__ void cp_async_wait_group()
+{
+    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+// Tiled TMA loads (2-D, 3-D) into this CTA's shared memory, completing on
+// `bar` (complete_tx).  `map` is the generic address of a tensor map in
+// kernel-parameter or global memory.  No multicast.
+__device__ __forceinline__ void tma_load_2d(void *dst, const void *map, int x, int y, uint64_t *bar)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::
+            "r"(smem_u32(dst)), "l"(map), "r"(x), "r"(y), "r"(smem_u32(bar))
+        : "memory");
+}
+
+__device__ __forceinline__ void tma_load_3d(void *dst, const void *map, int x, int y, int z, uint64_t *bar)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], [%5];" ::
+            "r"(smem_u32(dst)), "l"(map), "r"(x), "r"(y), "r"(z), "r"(smem_u32(bar))
+        : "memory");
+}
+
+// Tensor-map edits on the device: replace the global address of a map held
+// in shared memory (128-byte aligned), copy it to global memory with a
+// release of the tensormap proxy (warp-collective), and acquire it there
+// before the TMA loads that use it.
+__device__ __forceinline__ void tmap_replace_address(void *smap, const void *addr)
+{
+    asm volatile("tensormap.replace.tile.global_address.shared::cta.b1024.b64 [%0], %1;" ::"r"(smem_u32(smap)),
+                 "l"(addr)
+                 : "memory");
+}
+
+__device__ __forceinline__ void tmap_copy_release(void *gmap, const void *smap)
+{
+    asm volatile(
+        "tensormap.cp_fenceproxy.global.shared::cta.tensormap::generic.release.gpu.sync.aligned [%0], [%1], 128;" ::
+            "l"(gmap), "r"(smem_u32(smap))
+        : "memory");
+}
+
+__device__ __forceinline__ void tmap_acquire(const void *gmap)
+{
+    asm volatile("fence.proxy.tensormap::generic.acquire.gpu [%0], 128;" ::"l"(gmap) : "memory");
+}
+
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
@@ -233,6 +290,21 @@ __device__ __forceinline__ uint64_t umma_desc(const void *smem, uint32_t lbo, ui
     d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
     d |= (uint64_t)1 << 46;                  // descriptor version (sm_100)
     return d;                                 // base offset 0, layout type 0 (no swizzle)
+}
+
+// Shared-memory matrix descriptor, K-major with the 128-byte swizzle: rows of
+// 128 bytes (64 bf16 of K) as a TMA box with CU_TENSOR_MAP_SWIZZLE_128B writes
+// them, 8-row groups 1024 bytes apart, tile base 1024-byte aligned.  A K step
+// of 16 elements inside the 128-byte row advances the start address by 32.
+__device__ __forceinline__ uint64_t umma_desc_sw128(const void *smem)
+{
+    uint64_t d = 0;
+    d |= (uint64_t)((smem_u32(smem) >> 4) & 0x3FFFu);
+    d |= (uint64_t)1 << 16;                  // leading byte offset: unused here (16 bytes)
+    d |= (uint64_t)(1024u >> 4) << 32;       // stride byte offset: 8 rows x 128 bytes
+    d |= (uint64_t)1 << 46;                  // descriptor version (sm_100)
+    d |= (uint64_t)2 << 61;                  // layout type: 128-byte swizzle
+    return d;
 }
 
 // Instruction descriptor of kind::f16: bf16 A and B (K-major), f32 D, M x N.

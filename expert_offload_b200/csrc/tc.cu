@@ -12,6 +12,8 @@
 // gfx1151 engine README's self-written matrix-core GEMM for prefill
 // ("Windows" section); the Strata report, section "three counter-intuitive
 // conclusions": prefill is compute-bound, decode bandwidth-bound.
+#include <cuda.h>
+
 #include "device.cuh"
 #include "ptx.cuh"
 
@@ -20,30 +22,63 @@ namespace {
 
 constexpr int kM = 128;                    // weight rows per tile (MMA M)
 constexpr int kN = 128;                    // token pairs per tile (MMA N)
-constexpr int kKC = 128;                   // K per pipeline stage (8 MMAs of K = 16)
-constexpr int kQB = kKC / 32;              // 16-byte nibble quarters per row and chunk (4)
-constexpr int kTcThr = 512;                // 16 warps
-constexpr int kTcW = kTcThr / 32;
-constexpr int kTileBytes = kM * kKC * 2;   // one 128 x kKC bf16 operand tile
-constexpr uint32_t kLbo = (kM / 8) * 128;  // bytes between 8-element K chunks (2048)
-constexpr uint32_t kSbo = 128;             // bytes between 8-row groups
+constexpr int kKC = 64;                    // K per stage (4 MMAs of K = 16 per matrix)
+constexpr int kDqW = 16;                   // dequantising warps
+constexpr int kDqThr = kDqW * 32;
+constexpr int kMmaWarp = kDqW;             // issues the MMAs
+constexpr int kBWarp = kDqW + 1;           // TMA loads of the activation tiles
+constexpr int kRawWarp = kDqW + 2;         // TMA loads of the raw HFQ4 bytes
+constexpr int kTcThr = (kDqW + 3) * 32;
+constexpr int kTileBytes = kM * kKC * 2;   // one 128 x kKC bf16 operand tile (16 KB)
+constexpr uint32_t kLbo = (kM / 8) * 128;  // no-swizzle A tiles: bytes between 8-element K chunks
+constexpr uint32_t kSbo = 128;             // no-swizzle A tiles: bytes between 8-row groups
+constexpr int kRawW = 144;                 // staged bytes per weight row and HFQ4 block (16-byte window)
 constexpr uint32_t kTmemCols = 256;
+constexpr int kMaxTcCtas = 256;            // grid cap (one CTA per SM); sizes the tensor-map slots
+
+// Shared memory of one phase: two dequantised A buffers (gate [+ up]), a ring
+// of activation B tiles (TMA, 128-byte swizzle) and two raw buffers, each the
+// 144-byte window around one HFQ4 block of every weight row of the item.
+template <bool GU>
+struct TcCfg {
+    static constexpr int kRows = GU ? 2 * kM : kM;        // weight rows per item (gate rows, then up rows)
+    static constexpr int kBStages = GU ? 4 : 6;
+    static constexpr int kABytes = (GU ? 2 : 1) * kTileBytes;
+    static constexpr int kRawBytes = kRows * kRawW;
+    static constexpr int kBOff = 2 * kABytes;
+    static constexpr int kRawOff = kBOff + kBStages * kTileBytes;
+    static constexpr int kSmem = kRawOff + 2 * kRawBytes;
+    static constexpr int kDqWords = GU ? 4 : 2;             // nibble words a thread dequantises per stage
+    static_assert(kRows * 8 == kDqThr * kDqWords, "one dequantisation task per thread and stage");
+    static_assert(kBOff % 1024 == 0, "swizzled B tiles are 1024-byte aligned");
+};
+static_assert(TcCfg<true>::kSmem <= 227 * 1024 - 2048 && TcCfg<false>::kSmem <= 227 * 1024 - 2048,
+              "shared memory of the tensor-core kernels");
 
 struct TcArgs {
     const void *const *eptr;       // [E] expert base addresses
+    const uint8_t *eloc;           // [E] 0 = HBM, 1 = host-mapped, or null
     const int32_t *cnt, *off, *perm;
-    const float *wts;              // [T*k] routing weights, flat
-    const uint16_t *xin;           // gate/up: X_perm [T*k][H] or x [T][H]; down: H_perm [T*k][I] (bf16)
-    int x_direct;                  // gate/up reads row perm[q] / k of x instead of row q of X_perm
     uint16_t *hout;                // gate/up: H_perm out
     float *o;                      // down: O [T*k][H] f32, row q = pair perm[q]
     const int32_t *item_off;       // [E+1] prefix of work items of this phase
+    uint8_t *maps;                 // [CTAs][2][128] per-CTA tensor maps of the raw bytes (global)
     unsigned *status;
     long long timeout_ns;
+    unsigned long long *timeline;  // debug: [2 phases][64 stages][8] %globaltimer stamps of CTA 0, or null
     int E, H, I, k;
 };
 
-// Offset of element (row, kk) of a 128 x 64 operand tile in the canonical layout.
+constexpr int kTlStages = 64;
+
+// Debug timeline of CTA 0: stamp `s` of its stage c (first 64 stages).
+__device__ __forceinline__ void tl_stamp(const TcArgs &a, bool gu, int c, int s)
+{
+    if (a.timeline && blockIdx.x == 0 && c < kTlStages)
+        a.timeline[((gu ? 0 : 1) * kTlStages + c) * 8 + s] = globaltimer_ns();
+}
+
+// Offset of element (row, 8 * k8) of a no-swizzle 128 x kKC operand tile.
 __device__ __forceinline__ uint32_t tile_off(int row, int k8)
 {
     return (uint32_t)(row >> 3) * kSbo + (uint32_t)(row & 7) * 16u + (uint32_t)k8 * kLbo;
@@ -89,223 +124,286 @@ __device__ __forceinline__ uint4 deq8(uint32_t w, float scale, float zero)
     return make_uint4(r[0], r[1], r[2], r[3]);
 }
 
-__device__ bool tc_wait(const TcArgs &a, uint64_t *bar, uint32_t parity, int &abort)
+// Bounded wait for the phase of `bar` with the given parity.  Gives up when
+// another thread of the CTA has given up (*abort set) or at the deadline, when
+// it records HFQ_ERR_TIMEOUT and sets *abort.
+__device__ bool tc_wait(const TcArgs &a, uint64_t *bar, uint32_t parity, volatile int *abort)
 {
     uint64_t t0 = 0;
     for (int it = 0;; ++it) {
         if (mbar_try_wait(bar, parity)) return true;
+        if (abort && *abort) return false;
         if (it == 64) t0 = globaltimer_ns();
         if (it > 64 && (it & 15) == 0 && (long long)(globaltimer_ns() - t0) > a.timeout_ns) {
-            abort = 1;
+            if (abort) *abort = 1;
             atomicCAS(a.status, 0u, (unsigned)HFQ_ERR_TIMEOUT);
             return false;
         }
     }
 }
 
-// One persistent CTA per SM walks the work items (expert, row tile, token tile).
+// First byte of the 16-byte aligned 144-byte window around block b of a row
+// (rows are a whole, even number of blocks long, so the window stays inside
+// the row): an even block starts on 16 bytes, an odd one 8 bytes past.
+__device__ __forceinline__ int raw_window(int b) { return kBlockBytes * b - 8 * (b & 1); }
+
+// One persistent CTA per SM walks the work items (expert, row tile, token
+// tile) in K stages of 64.  Warp roles:
+//   raw warp   - per HFQ4 block of K, one 3-D TMA load of the 144-byte windows
+//                of all the item's weight rows (gate and up) into one of two
+//                raw buffers, through this CTA's copy of the raw tensor map,
+//                re-targeted to the item's expert (tensormap.replace)
+//   B warp     - per stage, one 2-D TMA load of the 128 x 64 activation tile
+//                (pair-ordered, 128-byte swizzle) into a ring of B tiles
+//   16 warps   - per stage, dequantise their rows' nibble words from the raw
+//                buffer into one of two A buffers; the item's epilogue
+//   MMA warp   - per stage, the MMAs of the A buffer against the B tile
+// Barriers (mbarriers): fullR/rfree per raw buffer, fullB/done per B tile,
+// aready per A buffer, tfree for the accumulators.  done[s] also frees the A
+// buffer of its stage.
 template <bool GU>
-__global__ void __launch_bounds__(kTcThr, 1) tc_kernel(const __grid_constant__ TcArgs a)
+__global__ void __launch_bounds__(kTcThr, 1)
+    tc_kernel(const __grid_constant__ TcArgs a, const __grid_constant__ CUtensorMap bmap,
+              const __grid_constant__ CUtensorMap rmap)
 {
+    using C = TcCfg<GU>;
+    constexpr int RB = C::kBStages;
     extern __shared__ __align__(1024) uint8_t smem[];
-    constexpr int kOps = GU ? 3 : 2;                 // operand tiles per stage (A0 [A1] B)
-    __shared__ uint64_t mma_bar[2];
+    __shared__ uint64_t fullB[RB], done_bar[RB], fullR[2], rfree[2], aready_bar[2], tfree_bar, fin_bar;
+    __shared__ alignas(128) uint8_t s_map[128];
     __shared__ uint32_t tmem_slot;
     __shared__ int s_abort;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int K = GU ? a.H : a.I, R = GU ? a.I : a.H;
-    const int rtiles = R / kM, nK = K / kKC;
+    const int K = GU ? a.H : a.I, Rr = GU ? a.I : a.H;
+    const int rtiles = Rr / kM, nK = K / kKC;
     const int rowB = (K + kBlock - 1) / kBlock * kBlockBytes;
     const size_t mg = (size_t)a.I * ((a.H + kBlock - 1) / kBlock) * kBlockBytes;
-    const uint32_t idesc = umma_idesc_bf16(kM, kN);
+    const int total = a.item_off[a.E];
+    const int my_items = total > (int)blockIdx.x ? (total - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
+    const int nchunks = my_items * nK;
+    volatile int *abortp = &s_abort;
 
     if (warp == 0) {
         tmem_alloc(&tmem_slot, kTmemCols);
         tmem_relinquish();
     }
     if (tid == 0) {
-        mbar_init(&mma_bar[0], 1);
-        mbar_init(&mma_bar[1], 1);
-        s_abort = 0;
+        for (int s = 0; s < RB; ++s) {
+            mbar_init(&fullB[s], 1);
+            mbar_init(&done_bar[s], 1);
+        }
+        for (int q = 0; q < 2; ++q) {
+            mbar_init(&fullR[q], 1);
+            mbar_init(&rfree[q], kDqW);
+            mbar_init(&aready_bar[q], kDqW);
+        }
+        mbar_init(&tfree_bar, kDqW);
+        mbar_init(&fin_bar, 1);
+        // the swizzled B tiles need a 1024-byte aligned base
+        s_abort = (smem_u32(smem) & 1023u) ? 1 : 0;
+        if (s_abort) atomicCAS(a.status, 0u, (unsigned)HFQ_ERR_CUDA);
         fence_mbar_init();
     }
+    if (warp == kRawWarp)   // this CTA's template of the raw tensor map
+        reinterpret_cast<uint32_t *>(s_map)[lane] = reinterpret_cast<const uint32_t *>(&rmap)[lane];
     tc_fence_before_sync();
     __syncthreads();
     tc_fence_after_sync();
     const uint32_t tmem = tmem_slot;
-    int abort = 0;
-    uint32_t commits[2] = {0u, 0u};
-    uint32_t chunk = 0;                              // stages used so far (buffer = chunk & 1)
-    const int total = a.item_off[a.E];
+    uint8_t *const abuf = smem;
+    uint8_t *const bbuf = smem + C::kBOff;
+    uint8_t *const rbuf = smem + C::kRawOff;
 
-    // Loads: a warp instruction reads 8 rows x 64 contiguous bytes (4 lanes
-    // of 16 bytes per row, rows fastest across lanes), and the 8 lanes of each
-    // shared-memory store phase write one 128-byte core-matrix column (8
-    // consecutive rows, one K chunk).  Weight rows: rid = (lane & 7) +
-    // 8 * (warp + kTcW * i), i < kRI (gate/up: rows >= 128 are the up
-    // matrix), quarter qq = lane >> 3.  Activation pieces: token n =
-    // (lane & 7) + 8 * (b & 15), K piece 4 * (b >> 4) + qq, b = warp + kTcW * i.
-    // The next chunk's loads (of this item or, at its last chunk, of the next
-    // item) are in flight while a chunk is dequantised and multiplied.
-    constexpr int kRI = (GU ? 2 * kM : kM) / (8 * kTcW);   // weight rows per thread and chunk
-    const int qq = lane >> 3, rl = lane & 7;
-    struct Geo {
-        int p0, nvalid, r0;
-        const uint8_t *gbase, *ubase;                // gate (or down) and up matrices
-        const uint16_t *xrow;                        // this thread's activation row, or null
+    // item -> (expert, first pair, valid pairs, first weight row)
+    struct Item {
+        int e, p0, nvalid, r0;
     };
-    static_assert(kTcW == 16, "one activation row per thread: n = (lane & 7) + 8 * warp");
-    const int xn = rl + 8 * warp;
-    auto geo_of = [&](int item) {
+    auto item_of = [&](int item) {
         int lo = 0, hi = a.E;                        // item_off[lo] <= item < item_off[lo + 1]
         while (hi - lo > 1) {
             const int mid = (lo + hi) >> 1;
             if (a.item_off[mid] <= item) lo = mid; else hi = mid;
         }
-        const int e = lo, local = item - a.item_off[e];
+        const int local = item - a.item_off[lo];
         const int rt = local % rtiles, nt = local / rtiles;
-        Geo g;
-        g.p0 = a.off[e] + nt * kN;
-        g.nvalid = min(kN, a.cnt[e] - nt * kN);
-        g.r0 = rt * kM;
-        const uint8_t *base = static_cast<const uint8_t *>(a.eptr[e]);
-        g.gbase = (GU ? base : base + 2 * mg) + (size_t)g.r0 * rowB;
-        g.ubase = base + mg + (size_t)g.r0 * rowB;
-        g.xrow = nullptr;
-        if (xn < g.nvalid) {
-            const int q = g.p0 + xn;
-            g.xrow = a.xin + (size_t)(GU && a.x_direct ? a.perm[q] / a.k : q) * K;
-        }
-        return g;
+        Item t;
+        t.e = lo;
+        t.p0 = a.off[lo] + nt * kN;
+        t.nvalid = min(kN, a.cnt[lo] - nt * kN);
+        t.r0 = rt * kM;
+        return t;
     };
-    float2 nsz[kRI];
-    uint4 nw[kRI];
-    uint4 nx[(kN * kKC / 8) / kTcThr];
-    auto load = [&](const Geo &g, int kc2) {
-        const int blk = (kc2 * kKC) / kBlock, sub = ((kc2 * kKC) % kBlock) / 2;   // nibble byte
-#pragma unroll
-        for (int i = 0; i < kRI; ++i) {
-            const int rid = rl + 8 * (warp + kTcW * i);
-            const uint8_t *rp = (GU && rid >= kM ? g.ubase : g.gbase) + (size_t)(rid & (kM - 1)) * rowB +
-                                (size_t)blk * kBlockBytes;
-            nsz[i] = __ldg(reinterpret_cast<const float2 *>(rp));
-            // the payload of an even block starts at 8 mod 16: two 8-byte loads
-            const uint2 lo = __ldg(reinterpret_cast<const uint2 *>(rp + 8 + sub + 16 * qq));
-            const uint2 hi = __ldg(reinterpret_cast<const uint2 *>(rp + 16 + sub + 16 * qq));
-            nw[i] = make_uint4(lo.x, lo.y, hi.x, hi.y);
-        }
-#pragma unroll
-        for (int i = 0; i < (kN * kKC / 8) / kTcThr; ++i) {
-            const int k8 = 4 * ((warp + kTcW * i) >> 4) + qq;
-            nx[i] = g.xrow ? __ldg(reinterpret_cast<const uint4 *>(g.xrow + kc2 * kKC + k8 * 8))
-                           : make_uint4(0u, 0u, 0u, 0u);
-        }
-    };
-    Geo cur{};
-    if ((int)blockIdx.x < total) {
-        cur = geo_of(blockIdx.x);
-        load(cur, 0);
-    }
-    for (int item = blockIdx.x; item < total; item += gridDim.x) {
-        const Geo g = cur;
-        const int p0 = g.p0, nvalid = g.nvalid, r0 = g.r0;
-        const int next = item + (int)gridDim.x;
-        Geo ng{};
-        if (next < total) ng = geo_of(next);
+    const int nb = (K + kBlock - 1) / kBlock;        // HFQ4 blocks (raw loads) per item
 
-        for (int kc = 0; kc < nK; ++kc, ++chunk) {
-            const int s = chunk & 1;
-            uint8_t *st = smem + (size_t)s * kOps * kTileBytes;
-            float2 sz[kRI];
-            uint4 w[kRI];
-            uint4 xv[(kN * kKC / 8) / kTcThr];
-#pragma unroll
-            for (int i = 0; i < kRI; ++i) { sz[i] = nsz[i]; w[i] = nw[i]; }
-#pragma unroll
-            for (int i = 0; i < (kN * kKC / 8) / kTcThr; ++i) xv[i] = nx[i];
-            if (!abort) {
-                if (kc + 1 < nK) load(g, kc + 1);
-                else if (next < total) load(ng, 0);
+    int issued = 0;
+    if (s_abort) {
+        // nothing runs
+    } else if (warp == kRawWarp) {
+        // ------------------------------------------------ raw HFQ4 bytes
+        uint8_t *gmap = a.maps + (size_t)blockIdx.x * 256;
+        int gs = 0;
+        for (int it = 0; it < my_items && !*abortp; ++it) {
+            const Item t = item_of((int)blockIdx.x + it * (int)gridDim.x);
+            const uint8_t *base = static_cast<const uint8_t *>(a.eptr[t.e]) + (GU ? 0 : 2 * mg);
+            const bool host = a.eloc && a.eloc[t.e];
+            uint8_t *slot = gmap + (it & 1) * 128;
+            if (!host) {
+                if (lane == 0) tmap_replace_address(s_map, base);
+                __syncwarp();
+                tmap_copy_release(slot, s_map);
+                if (lane == 0) tmap_acquire(slot);
             }
-            if (commits[s] && !abort) tc_wait(a, &mma_bar[s], (commits[s] - 1) & 1, abort);
-            if (!abort) {
-                // weights: row rid, K pieces 4 qq .. 4 qq + 3 of this chunk
-#pragma unroll
-                for (int i = 0; i < kRI; ++i) {
-                    const int rid = rl + 8 * (warp + kTcW * i);
-                    uint8_t *dst = st + (GU && rid >= kM ? kTileBytes : 0);
-                    const int rr = rid & (kM - 1);
-                    *reinterpret_cast<uint4 *>(dst + tile_off(rr, 4 * qq + 0)) = deq8(w[i].x, sz[i].x, sz[i].y);
-                    *reinterpret_cast<uint4 *>(dst + tile_off(rr, 4 * qq + 1)) = deq8(w[i].y, sz[i].x, sz[i].y);
-                    *reinterpret_cast<uint4 *>(dst + tile_off(rr, 4 * qq + 2)) = deq8(w[i].z, sz[i].x, sz[i].y);
-                    *reinterpret_cast<uint4 *>(dst + tile_off(rr, 4 * qq + 3)) = deq8(w[i].w, sz[i].x, sz[i].y);
-                }
-                // activations: 128 token rows x kKC values, 16 bytes per piece
-                uint8_t *bt = st + (size_t)(kOps - 1) * kTileBytes;
-#pragma unroll
-                for (int i = 0; i < (kN * kKC / 8) / kTcThr; ++i) {
-                    const int blkid = warp + kTcW * i;
-                    const int n = rl + 8 * (blkid & 15), k8 = 4 * (blkid >> 4) + qq;
-                    *reinterpret_cast<uint4 *>(bt + tile_off(n, k8)) = xv[i];
+            for (int b = 0; b < nb && !*abortp; ++b, ++gs) {
+                const int q = gs & 1;
+                if (gs >= 2 && !tc_wait(a, &rfree[q], (uint32_t)((gs >> 1) - 1) & 1u, abortp)) break;
+                uint8_t *dst = rbuf + q * C::kRawBytes;
+                if (!host) {
+                    if (lane == 0) {
+                        mbar_arrive_expect_tx(&fullR[q], (uint32_t)C::kRawBytes);
+                        if (GU) tma_load_3d(dst, slot, raw_window(b), t.r0, 0, &fullR[q]);
+                        else tma_load_2d(dst, slot, raw_window(b), t.r0, &fullR[q]);
+                    }
+                } else {
+                    // host-mapped expert: plain 16-byte loads over PCIe
+                    for (int i = lane; i < C::kRows * (kRawW / 16); i += 32) {
+                        const int row = i / (kRawW / 16), piece = i - row * (kRawW / 16);
+                        const uint8_t *src = base + (GU && row >= kM ? mg : 0) +
+                                             (size_t)(t.r0 + (row & (kM - 1))) * rowB + raw_window(b) + 16 * piece;
+                        *reinterpret_cast<uint4 *>(dst + row * kRawW + 16 * piece) = __ldcv(reinterpret_cast<const uint4 *>(src));
+                    }
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&fullR[q]);
                 }
             }
-            fence_proxy_async_smem();
-            __syncthreads();
-            if (tid == 0 && !abort && !s_abort) {
-                tc_fence_after_sync();
-                const uint8_t *bt = st + (size_t)(kOps - 1) * kTileBytes;
+        }
+        // an aborted CTA still lets its last raw loads land before it ends
+        // (each buffer holds at most one load in flight)
+        if (lane == 0)
+            for (int g = max(0, gs - 2); g < gs; ++g) tc_wait(a, &fullR[g & 1], (uint32_t)(g >> 1) & 1u, nullptr);
+    } else if (warp == kBWarp) {
+        // ------------------------------------------------ activation tiles
+        int p0 = 0, nb_issued = 0;
+        for (int c = 0; c < nchunks; ++c) {
+            const int it = c / nK, kc = c - it * nK;
+            if (kc == 0) p0 = item_of((int)blockIdx.x + it * (int)gridDim.x).p0;
+            if (c >= RB && !tc_wait(a, &done_bar[(c - RB) % RB], (uint32_t)((c - RB) / RB) & 1u, abortp)) break;
+            if (lane == 0) {
+                mbar_arrive_expect_tx(&fullB[c % RB], (uint32_t)kTileBytes);
+                tma_load_2d(bbuf + (c % RB) * kTileBytes, &bmap, kc * kKC, p0, &fullB[c % RB]);
+            }
+            nb_issued = c + 1;
+            __syncwarp();
+        }
+        // an aborted CTA still lets its last activation loads land
+        if (lane == 0)
+            for (int c = max(0, nb_issued - RB); c < nb_issued; ++c)
+                tc_wait(a, &fullB[c % RB], (uint32_t)(c / RB) & 1u, nullptr);
+    } else if (warp == kMmaWarp) {
+        // ------------------------------------------------ MMA issue
+        const uint32_t idesc = umma_idesc_bf16(kM, kN);
+        for (int c = 0; c < nchunks; ++c) {
+            const int it = c / nK, kc = c - it * nK;
+            if (kc == 0 && it > 0 && !tc_wait(a, &tfree_bar, (uint32_t)(it - 1) & 1u, abortp)) break;
+            if (!tc_wait(a, &aready_bar[c & 1], (uint32_t)(c >> 1) & 1u, abortp)) break;
+            if (!tc_wait(a, &fullB[c % RB], (uint32_t)(c / RB) & 1u, abortp)) break;
+            tc_fence_after_sync();
+            if (lane == 0) tl_stamp(a, GU, c, 5);
+            if (lane == 0) {
+                // the A tile was written through the generic proxy by other
+                // threads and released to this one by aready; this proxy
+                // fence orders it before the MMAs' async-proxy reads
+                fence_proxy_async_smem();
+                const uint8_t *A = abuf + (c & 1) * C::kABytes;
+                const uint8_t *B = bbuf + (c % RB) * kTileBytes;
 #pragma unroll
                 for (int ks = 0; ks < kKC / 16; ++ks) {
-                    const uint64_t bd = umma_desc(bt + 2 * ks * kLbo, kLbo, kSbo);
-                    umma_bf16(tmem, umma_desc(st + 2 * ks * kLbo, kLbo, kSbo), bd, idesc,
-                              (kc | ks) != 0);
+                    const uint64_t bd = umma_desc_sw128(B + 32 * ks);
+                    umma_bf16(tmem, umma_desc(A + 2 * ks * kLbo, kLbo, kSbo), bd, idesc, (kc | ks) != 0);
                     if (GU)
-                        umma_bf16(tmem + kN, umma_desc(st + kTileBytes + 2 * ks * kLbo, kLbo, kSbo),
-                                  bd, idesc, (kc | ks) != 0);
+                        umma_bf16(tmem + kN, umma_desc(A + kTileBytes + 2 * ks * kLbo, kLbo, kSbo), bd,
+                                  idesc, (kc | ks) != 0);
                 }
-                umma_commit(&mma_bar[s]);
+                umma_commit(&done_bar[c % RB]);
+                tl_stamp(a, GU, c, 6);
             }
-            ++commits[s];
-            if (abort && tid == 0) s_abort = 1;
+            ++issued;
+            __syncwarp();
         }
-        // all MMAs of the item are complete once its last commit has arrived
-        const int sl = (chunk - 1) & 1;
-        if (!abort && !s_abort) tc_wait(a, &mma_bar[sl], (commits[sl] - 1) & 1, abort);
-        tc_fence_after_sync();
-        if (!abort && !s_abort) {
-            constexpr int kCols = kN / (kTcW / 4);                // columns per warp
-            const int lg = warp & 3, half = warp >> 2;          // TMEM lane group, column group
-            const int r = lg * 32 + lane;
-            const uint32_t trow = tmem + ((uint32_t)(lg * 32) << 16);
+    } else {
+        // ------------------------------------------------ dequantisation
+        // task: weight row drow, nibble words dw0 .. dw0 + kDqWords - 1 of the
+        // stage (each 8-lane phase stores one 128-byte core-matrix column)
+        const int drow = GU ? (lane & 7) + 8 * ((lane >> 3) + 4 * (warp >> 1))
+                            : (lane & 7) + 8 * ((lane >> 3) + 4 * (warp >> 2));
+        const int dw0 = GU ? 4 * (warp & 1) : 2 * (warp & 3);
+        uint8_t *const adst0 = abuf + (GU && drow >= kM ? kTileBytes : 0) + tile_off(drow & (kM - 1), 0);
+        int gs = -1;
 #pragma unroll 1
-            for (int c = half * kCols; c < (half + 1) * kCols; c += 16) {
-                float g[16], u[16];
-                tmem_ld16(trow + c, g);
-                if (GU) tmem_ld16(trow + kN + c, u);
-                tmem_ld_wait();
+        for (int c = 0; c < nchunks; ++c) {
+            const int it = c / nK, kc = c - it * nK;
+            const int j = kc & 3, b = kc >> 2;
+            const bool tl = tid == 0;
+            if (tl) tl_stamp(a, GU, c, 0);
+            if (j == 0) ++gs;                         // the stage opens a new raw buffer (HFQ4 block)
+            if (j == 0 && !tc_wait(a, &fullR[gs & 1], (uint32_t)(gs >> 1) & 1u, abortp)) break;
+            if (tl) tl_stamp(a, GU, c, 1);
+            // the MMAs of stage c - 2 are done: its A buffer is free
+            if (c >= 2 && !tc_wait(a, &done_bar[(c - 2) % RB], (uint32_t)((c - 2) / RB) & 1u, abortp)) break;
+            if (tl) tl_stamp(a, GU, c, 2);
+            const uint8_t *raw = rbuf + (gs & 1) * C::kRawBytes + drow * kRawW + 8 * (b & 1);
+            const float2 sz = *reinterpret_cast<const float2 *>(raw);
+            const uint8_t *pw = raw + 8 + 32 * j + 4 * dw0;
+            uint8_t *ad = adst0 + (c & 1) * C::kABytes;
 #pragma unroll
-                for (int j = 0; j < 16; ++j) {
-                    const int n = c + j;
-                    if (n >= nvalid) break;
-                    const int p = p0 + n;
-                    if (GU) {
-                        a.hout[(size_t)p * a.I + r0 + r] = float_to_bf16_bits(silu(g[j]) * u[j]);
-                    } else {
-                        a.o[(size_t)p * a.H + r0 + r] = g[j];
+            for (int h = 0; h < C::kDqWords / 2; ++h) {
+                const uint2 w = *reinterpret_cast<const uint2 *>(pw + 8 * h);
+                *reinterpret_cast<uint4 *>(ad + (dw0 + 2 * h) * kLbo) = deq8(w.x, sz.x, sz.y);
+                *reinterpret_cast<uint4 *>(ad + (dw0 + 2 * h + 1) * kLbo) = deq8(w.y, sz.x, sz.y);
+            }
+            __syncwarp();
+            if (lane == 0) {
+                mbar_arrive(&aready_bar[c & 1]);
+                if (j == 3 || kc == nK - 1) mbar_arrive(&rfree[gs & 1]);   // raw buffer read
+            }
+            if (tl) tl_stamp(a, GU, c, 3);
+
+            if (kc == nK - 1) {
+                // epilogue: warp w reads TMEM lanes 32 (w % 4) .. + 31 (weight
+                // rows), columns (token pairs) 32 (w / 4) .. + 31
+                if (!tc_wait(a, &done_bar[c % RB], (uint32_t)(c / RB) & 1u, abortp)) break;
+                tc_fence_after_sync();
+                const Item t = item_of((int)blockIdx.x + it * (int)gridDim.x);
+                const int lg = warp & 3, cgp = warp >> 2;
+                const int r = lg * 32 + lane;
+                const uint32_t trow = tmem + ((uint32_t)(lg * 32) << 16);
+#pragma unroll 1
+                for (int col = cgp * 32; col < cgp * 32 + 32; col += 16) {
+                    float g[16], u[16];
+                    tmem_ld16(trow + col, g);
+                    if (GU) tmem_ld16(trow + kN + col, u);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int jj = 0; jj < 16; ++jj) {
+                        const int n = col + jj;
+                        if (n >= t.nvalid) break;
+                        const int p = t.p0 + n;
+                        if (GU)
+                            a.hout[(size_t)p * a.I + t.r0 + r] = float_to_bf16_bits(silu(g[jj]) * u[jj]);
+                        else
+                            a.o[(size_t)p * a.H + t.r0 + r] = g[jj];
                     }
                 }
+                tc_fence_before_sync();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&tfree_bar);
             }
         }
-        tc_fence_before_sync();
-        __syncthreads();
-        if (s_abort) abort = 1;
-        cur = ng;
     }
-    // no MMA may still write tensor memory when it is freed
-    if (tid == 0 && chunk) {
-        const int sl = (chunk - 1) & 1;
-        int dummy = 0;
-        tc_wait(a, &mma_bar[sl], (commits[sl] - 1) & 1, dummy);
+    // no MMA may still write tensor memory, nor a TMA load shared memory,
+    // when the CTA ends
+    if (warp == kMmaWarp && lane == 0 && issued > 0) {
+        umma_commit(&fin_bar);
+        tc_wait(a, &fin_bar, 0u, nullptr);
     }
     tc_fence_before_sync();
     __syncthreads();
@@ -333,13 +431,6 @@ __global__ void tc_plan_kernel(const int32_t *__restrict__ cnt, int E, int I, in
         }
         gu_off[E] = a; dn_off[E] = b;
     }
-}
-
-// pos[perm[q]] = q (the gate/up kernel reads bf16 x through perm itself).
-__global__ void tc_pos_kernel(const int32_t *__restrict__ perm, int P, int32_t *__restrict__ pos)
-{
-    for (int q = blockIdx.x * blockDim.x + threadIdx.x; q < P; q += gridDim.x * blockDim.x)
-        pos[perm[q]] = q;
 }
 
 // X_perm[q] = x[token of pair perm[q]] as bf16 (16 bytes per thread step);
@@ -404,6 +495,7 @@ int tc_sms()
         int dev = 0;
         cudaGetDevice(&dev);
         cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+        n = std::min(n, kMaxTcCtas);
     }
     return n;
 }
@@ -414,13 +506,62 @@ size_t tc_workspace_bytes(int T, int k, int H, int I, int E)
 {
     const size_t P = (size_t)T * k;
     auto r256 = [](size_t b) { return (b + 255) / 256 * 256; };
-    return r256(P * H * 2) + r256(P * I * 2) + 2 * r256((size_t)(E + 1) * 4) + r256(P * H * 4) + r256(P * 4);
+    return r256(P * H * 2) + r256(P * I * 2) + 2 * r256((size_t)(E + 1) * 4) + r256(P * H * 4) + r256(P * 4) +
+           r256((size_t)kMaxTcCtas * 256);
 }
 
+// Rows of whole HFQ4 blocks must be a multiple of 16 bytes (an even number of
+// blocks) for the tensor maps of the raw bytes; tiles are 128 rows.
 bool tc_supported(int H, int I)
 {
-    return H % kM == 0 && I % kM == 0 && H % kKC == 0 && I % kKC == 0;
+    const int nbh = (H + kBlock - 1) / kBlock, nbi = (I + kBlock - 1) / kBlock;
+    return H % kM == 0 && I % kM == 0 && nbh % 2 == 0 && nbi % 2 == 0;
 }
+
+namespace {
+
+using EncodeTiled = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                 const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                 CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiled encode_fn()
+{
+    static EncodeTiled fn = nullptr;
+    if (!fn) {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiled>(p);
+    }
+    return fn;
+}
+
+// bf16 [rows][K] (pair-ordered activations or h): 128 x 64 boxes, 128-byte swizzle.
+bool encode_act(CUtensorMap *m, const void *base, int K, size_t rows)
+{
+    const cuuint64_t dim[2] = {(cuuint64_t)K, (cuuint64_t)rows};
+    const cuuint64_t stride[1] = {(cuuint64_t)K * 2};
+    const cuuint32_t box[2] = {(cuuint32_t)kKC, (cuuint32_t)kN}, es[2] = {1, 1};
+    return encode_fn()(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dim, stride, box, es,
+                       CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                       CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Raw HFQ4 bytes of one expert: gate/up as [2][I][rowB] (up = gate + mg), down
+// as [H][rowB]; 144-byte x 128-row boxes (x 2 matrices).  `base` is a
+// placeholder: the kernel re-targets a copy of the map to each item's expert.
+bool encode_raw(CUtensorMap *m, const void *base, bool gu, int rows, int rowB, size_t mg)
+{
+    const cuuint64_t dim[3] = {(cuuint64_t)rowB, (cuuint64_t)rows, 2};
+    const cuuint64_t stride[2] = {(cuuint64_t)rowB, (cuuint64_t)mg};
+    const cuuint32_t box[3] = {(cuuint32_t)kRawW, (cuuint32_t)kM, 2}, es[3] = {1, 1, 1};
+    return encode_fn()(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, gu ? 3 : 2, const_cast<void *>(base), dim, stride, box,
+                       es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                       CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
 
 hfq_status launch_tc(const hfq4_layer &L, const void *x, bool x_f32, int T, int k, const int32_t *cnt,
                      const int32_t *off, const int32_t *perm, const float *wts, float *y,
@@ -442,30 +583,37 @@ hfq_status launch_tc(const hfq4_layer &L, const void *x, bool x_f32, int T, int 
     float *ob = reinterpret_cast<float *>(w);
     w += r256(P * H * 4);
     int32_t *pos = reinterpret_cast<int32_t *>(w);
+    w += r256(P * 4);
+    uint8_t *maps = w;
+
+    if (!encode_fn()) return fail(HFQ_ERR_CUDA, "tensor-core path: cuTensorMapEncodeTiled unavailable");
+    const int rowB_gu = (H + kBlock - 1) / kBlock * kBlockBytes, rowB_dn = (I + kBlock - 1) / kBlock * kBlockBytes;
+    const size_t mg = (size_t)I * rowB_gu;
+    CUtensorMap xmap, hmap, rmap_gu, rmap_dn;
+    if (!encode_act(&xmap, xp, H, P) || !encode_act(&hmap, hp, I, P) ||
+        !encode_raw(&rmap_gu, maps, true, I, rowB_gu, mg) || !encode_raw(&rmap_dn, maps, false, H, rowB_dn, mg))
+        return fail(HFQ_ERR_CUDA, "tensor-core path: tensor map encoding failed (H %d, I %d, pairs %zu)", H, I, P);
 
     static bool attr = false;
-    const int smem_gu = 2 * 3 * kTileBytes, smem_dn = 2 * 2 * kTileBytes;
+    const int smem_gu = TcCfg<true>::kSmem, smem_dn = TcCfg<false>::kSmem;
     if (!attr) {
         cudaFuncSetAttribute(tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_gu);
         cudaFuncSetAttribute(tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_dn);
         attr = true;
     }
     tc_plan_kernel<<<1, 512, 0, s>>>(cnt, E, I, H, gu_off, dn_off);
+    // pair-ordered bf16 activations (the TMA tiles need contiguous rows)
     const size_t n8 = P * H / 8;
-    if (x_f32)
-        tc_gather_kernel<<<(unsigned)std::min<size_t>((n8 + 255) / 256, (size_t)tc_sms() * 16), 256, 0, s>>>(
-            x, 1, perm, (int)P, k, H, xp, pos);
-    else
-        tc_pos_kernel<<<(unsigned)std::min<size_t>((P + 255) / 256, (size_t)tc_sms() * 4), 256, 0, s>>>(
-            perm, (int)P, pos);
+    tc_gather_kernel<<<(unsigned)std::min<size_t>((n8 + 255) / 256, (size_t)tc_sms() * 16), 256, 0, s>>>(
+        x, x_f32 ? 1 : 0, perm, (int)P, k, H, xp, pos);
     TcArgs a;
-    a.eptr = L.expert_ptr; a.cnt = cnt; a.off = off; a.perm = perm; a.wts = wts;
-    a.status = status; a.timeout_ns = timeout_ns; a.E = E; a.H = H; a.I = I; a.k = k;
-    a.xin = x_f32 ? xp : static_cast<const uint16_t *>(x); a.x_direct = x_f32 ? 0 : 1;
+    a.eptr = L.expert_ptr; a.eloc = L.expert_loc; a.cnt = cnt; a.off = off; a.perm = perm;
+    a.maps = maps; a.status = status; a.timeout_ns = timeout_ns; a.E = E; a.H = H; a.I = I; a.k = k;
+    a.timeline = static_cast<unsigned long long *>(option_timeline());
     a.hout = hp; a.o = nullptr; a.item_off = gu_off;
-    tc_kernel<true><<<tc_sms(), kTcThr, smem_gu, s>>>(a);
-    a.xin = hp; a.x_direct = 0; a.hout = nullptr; a.o = ob; a.item_off = dn_off;
-    tc_kernel<false><<<tc_sms(), kTcThr, smem_dn, s>>>(a);
+    tc_kernel<true><<<tc_sms(), kTcThr, smem_gu, s>>>(a, xmap, rmap_gu);
+    a.hout = nullptr; a.o = ob; a.item_off = dn_off;
+    tc_kernel<false><<<tc_sms(), kTcThr, smem_dn, s>>>(a, hmap, rmap_dn);
     const size_t n4 = (size_t)T * H / 4;
     tc_combine_kernel<<<(unsigned)std::min<size_t>((n4 + 255) / 256, (size_t)tc_sms() * 16), 256, 0, s>>>(
         ob, pos, wts, T, k, H, y, y_bf16);

@@ -169,8 +169,12 @@ typedef struct {
  *           HFQ_PATH_TC; with AUTO and T > 8 they select the tensor-core
  *           path, without them T > 8 runs the per-layer GEMV kernels.
  *   path:   AUTO: T <= 8 -> persistent GEMV kernel; T > 8 with grouping ->
- *           tensor cores.  GEMV forces CUDA cores; TC forces the tensor-core
- *           path [WMMA]: weights dequantised to RN_bf16(fmaf(scale, q, zero)),
+ *           tensor cores where the shape allows them (hidden and inter
+ *           multiples of 128, each with an even number of 256-weight blocks
+ *           per row, so that rows are whole 16-byte units for the tensor
+ *           maps), else the per-layer GEMV kernels.  GEMV forces CUDA cores;
+ *           TC forces the tensor-core path (HFQ_ERR_UNSUPPORTED for other
+ *           shapes) [WMMA]: weights dequantised to RN_bf16(fmaf(scale, q, zero)),
  *           x rounded to bf16 (exact for bf16 input), f32 accumulation, h
  *           rounded to bf16 before the down projection, each pair's down
  *           output kept in f32 and y summed over the k slots in slot order

@@ -2,7 +2,8 @@
 not multiples of the 256-weight HFQ4 block (rows padded to whole blocks, pad
 elements stored as q = 0 and counting as zero), through every path the
 forward takes for them: the persistent kernels (1..8 tokens), the per-layer
-GEMV kernels and the tensor-core path (40 tokens)."""
+GEMV kernels (40 tokens) and the tensor-core path (40 and 300 tokens, with
+rows of an even number of blocks)."""
 import dataclasses
 
 import numpy as np
@@ -85,7 +86,7 @@ def test_ragged_persistent_kernels(eo, ragged, T):
     assert err <= TOL, err
 
 
-def test_ragged_gemv_and_tensor_core_paths(eo, ragged):
+def test_ragged_gemv_path(eo, ragged):
     w, store = ragged
     H, I, E, k, T = w.hidden, w.inter, w.experts, w.top_k, 40
     logits = W.zipf_logits(w, 0, 300, T)
@@ -96,6 +97,45 @@ def test_ragged_gemv_and_tensor_core_paths(eo, ragged):
     y_gv = _forward(eo, store.layers[0], x, T, k, routed, eo.PATH_GEMV, H, I, E, grouped=False)
     ref_exact = moe.moe_layer(moe.ExpertCache(OraclePackedLayer(w, 0), H, I), H, I, xv, ridx, rw)
     assert max_rel_err(y_gv, ref_exact) <= TOL
+
+
+def test_ragged_shape_without_whole_16_byte_rows_refuses_the_tensor_cores(eo, ragged):
+    """inter 640 = 3 blocks per down row (408 bytes): no tensor map can step
+    over such rows, so a forced tensor-core call is refused and AUTO takes the
+    GEMV kernels."""
+    w, store = ragged
+    H, I, E, k, T = w.hidden, w.inter, w.experts, w.top_k, 40
+    x, _ = W.activations(w, 300, T)
+    routed = _route(eo, W.zipf_logits(w, 0, 300, T), k)
+    with pytest.raises(Exception, match="even number"):
+        _forward(eo, store.layers[0], x, T, k, routed, eo.PATH_TC, H, I, E, grouped=True)
+    y = _forward(eo, store.layers[0], x, T, k, routed, eo.PATH_AUTO, H, I, E, grouped=True)
+    ridx, rw = route.route(W.zipf_logits(w, 0, 300, T), k)
+    ref = moe.moe_layer(moe.ExpertCache(OraclePackedLayer(w, 0), H, I), H, I,
+                        synth.bf16_bits_to_f32(x).astype(np.float64), ridx, rw)
+    assert max_rel_err(y, ref) <= TOL
+
+
+@pytest.fixture(scope="module")
+def ragged_tc(eo):
+    """16 experts, hidden 384 (1.5 blocks per gate/up row, padded to 2),
+    intermediate 896 (3.5 blocks per down row, padded to 4): partial K
+    blocks and a partial last raw load on the tensor-core path."""
+    from expert_offload_b200.model import ExpertStore
+    w = dataclasses.replace(W.WORKLOADS[4], hidden=384, inter=896, experts=16, top_k=4)
+    store = ExpertStore(torch, 1, w.experts, w.hidden, w.inter, device_fill(torch, w))
+    return w, store
+
+
+@pytest.mark.parametrize("T", [40, 300])
+def test_ragged_tensor_core_path(eo, ragged_tc, T):
+    w, store = ragged_tc
+    H, I, E, k = w.hidden, w.inter, w.experts, w.top_k
+    logits = W.zipf_logits(w, 0, 300, T)
+    x, _ = W.activations(w, 300, T)
+    routed = _route(eo, logits, k)
+    ridx, rw = route.route(logits, k)
+    xv = synth.bf16_bits_to_f32(x).astype(np.float64)
     y_tc = _forward(eo, store.layers[0], x, T, k, routed, eo.PATH_TC, H, I, E, grouped=True)
     ref_tc = moe.moe_layer(moe.ExpertCache(OraclePackedLayer(w, 0), H, I, tc=True), H, I, xv, ridx, rw)
     err = max_rel_err(y_tc, ref_tc)

@@ -97,6 +97,34 @@ def test_tc_and_gemv_paths_agree(eo, small_layer):
     assert max_rel_err(y_tc, ref_exact) <= 2e-2
 
 
+def test_tc_path_with_host_mapped_experts(eo):
+    """Every other expert in pinned host memory: the tensor-core kernels read
+    those experts' bytes with plain loads over PCIe instead of TMA tiles and
+    must give the same layer."""
+    from expert_offload_b200.model import ExpertStore
+    w = dataclasses.replace(W.WORKLOADS[4], experts=16)
+    H, I, E, k, T = w.hidden, w.inter, w.experts, w.top_k, 96
+    loc = (np.arange(E) % 2).astype(np.uint8)[None, :]
+    slot = np.zeros((1, E), np.int64)
+    for where in (0, 1):
+        ids = np.nonzero(loc[0] == where)[0]
+        slot[0, ids] = np.arange(len(ids))
+    store = ExpertStore(torch, 1, E, H, I, device_fill(torch, w), loc=loc, slot=slot)
+    try:
+        logits = W.zipf_logits(w, 0, 700, T)
+        x, _ = W.activations(w, 700, T)
+        routed = _route(eo, logits, k)
+        y = _forward(eo, store.layers[0], x, T, k, routed, eo.PATH_TC, H, I, E)
+        ridx, rw = route.route(logits, k)
+        assert set(ridx.ravel() % 2) == {0, 1}          # experts from both memories
+        cache = moe.ExpertCache(OraclePackedLayer(w, 0), H, I, tc=True)
+        ref = moe.moe_layer(cache, H, I, synth.bf16_bits_to_f32(x).astype(np.float64), ridx, rw)
+        err = max_rel_err(y, ref)
+        assert err <= TOL, err
+    finally:
+        store.close()
+
+
 @pytest.mark.slow
 def test_tc_prefill_chunk_8192_sampled(eo):
     """The 512-expert, 8192-token prefill chunk at full size; the oracle checks
