@@ -16,12 +16,18 @@
 //      layer input meanwhile.
 //   2. warp w computes the gate/up rows of slot w (and w + 8) as soon as that
 //      slot has landed: nibbles decoded in registers, warp-shuffle sums,
-//      h = silu(g) * u into an L2-resident buffer.
-//   3. once a release counter shows every CTA's h rows written, warp w takes
-//      its slot's down rows against the full h, times the routing weight; the
-//      eight warps' sums are added in a fixed order, the bf16 residual is
-//      applied, and the CTA's rows of the next layer input are written.
-//   4. a grid-wide barrier ends the layer.
+//      h = silu(g) * u into an L2-resident buffer as 8-byte {value, tag}
+//      words, the tag naming this launch and layer.
+//   3. warp w polls its slot's h words until every tag is this layer's (one
+//      64-bit access reads a value with its tag, so no fence or counter is
+//      needed), takes its slot's down rows against the full h, times the
+//      routing weight; the eight warps' sums are added in a fixed order, the
+//      bf16 residual is applied, and the CTA's rows of the next layer input
+//      are written as tagged words too.
+//   4. the next layer starts once this CTA has read every row of its input
+//      with the next layer's tag, i.e. once every CTA has finished this one
+//      (no separate grid barrier; h and x are double-buffered by layer
+//      parity, which that ordering makes safe).
 // The expert address table of layer l+1 comes into shared memory (cp.async)
 // while layer l runs.  Every wait is bounded (sync.cuh); on expiry the status
 // word holds HFQ_ERR_TIMEOUT and every CTA winds down.
@@ -54,8 +60,8 @@ struct D1Args {
     const float *wts_in;
     const void *x0;           // [H] bf16 (f32 when x0_f32)
     uint16_t *x_out;          // [H] bf16 input of the layer after the last, or null
-    uint16_t *xbuf;           // [2][H] bf16 ping-pong between layers (L > 1)
-    float *h;                 // [k][Ip]
+    uint64_t *xbuf;           // [2][H] {bf16 value, tag} words, ping-pong between layers (L > 1)
+    uint64_t *h;              // [2][k][Ip] {f32 value, tag} words, ping-pong between layers
     float *y;                 // [L][H], or null
     uint16_t *y_bf16;         // [H] of the last layer, or null
     int32_t *idx_all;         // [L][k], or null
@@ -82,6 +88,28 @@ struct D1Shared {
     int last_cta;
     int armed;                        // layers whose slot barriers were armed
 };
+
+// Exchange tag of layer l (< 64) in launch `epoch`: never 0 (a fresh
+// workspace), and as f32 a signalling NaN, which no h value that another
+// kernel leaves in the buffer is.  Every launch rewrites every h word it reads
+// at every layer, so a word holds this launch's previous layer or the last
+// layer of an earlier launch, never a matching tag, whatever the epoch's wrap.
+__device__ __forceinline__ uint32_t xch_tag(uint32_t epoch, int l)
+{
+    return 0x7FA00000u | ((epoch & 0x1FFFu) << 7) | (uint32_t)(l + 1);
+}
+
+__device__ __forceinline__ void st_tagged(uint64_t *p, float v, uint32_t tag)
+{
+    const uint64_t w = (uint64_t)__float_as_uint(v) | ((uint64_t)tag << 32);
+    asm volatile("st.relaxed.gpu.global.b64 [%0], %1;" ::"l"(p), "l"(w) : "memory");
+}
+
+// Two tagged words (16-byte aligned); each 64-bit element is read atomically.
+__device__ __forceinline__ void ld_tagged2(const uint64_t *p, uint64_t &a, uint64_t &b)
+{
+    asm volatile("ld.relaxed.gpu.global.v2.b64 {%0, %1}, [%2];" : "=l"(a), "=l"(b) : "l"(p) : "memory");
+}
 
 // Padded f32 column of activation c in shared memory: 4 floats after every 64,
 // so the lanes' 64-wide slices start on distinct bank quads and stay 16-byte
@@ -182,6 +210,7 @@ __global__ void __launch_bounds__(kThr, 1) decode1_kernel(const __grid_constant_
     float *ysh = reinterpret_cast<float *>(smem + a.ysh_off);        // [kW][kMaxDRows]
     D1Shared &sh = *reinterpret_cast<D1Shared *>(smem + a.sh_off);
     const WaitCtx wc{a.ctl, a.timeout_ns, &sh.abort};
+    const uint32_t epoch = *(volatile const unsigned *)(a.ctl + kCtlEpoch);
 
     if (tid == 0) {
         for (int j = 0; j < kMaxK; ++j) {
@@ -199,6 +228,63 @@ __global__ void __launch_bounds__(kThr, 1) decode1_kernel(const __grid_constant_
     for (int l = 0; l < a.L; ++l) {
         stamp(a, l, 0);
         const uint32_t par = l & 1;          // parity of this layer's slot-barrier phases
+        // ---------------------------------------------- 1a. layer input -> xs
+        if (l == 0) {
+            const bool f32 = a.x0_f32;
+            const int per = f32 ? 4 : 8;                // values per 16-byte load
+            const int nld = H / per;
+            for (int i = tid; i < nld; i += kThr) {
+                const uint4 v = __ldcg(static_cast<const uint4 *>(a.x0) + i);
+                float2 *dst = reinterpret_cast<float2 *>(xs + xp4(i * per));
+                if (f32) {
+                    dst[0] = make_float2(__uint_as_float(v.x), __uint_as_float(v.y));
+                    dst[1] = make_float2(__uint_as_float(v.z), __uint_as_float(v.w));
+                } else {
+                    const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                    for (int r = 0; r < 4; ++r)
+                        dst[r] = make_float2(__uint_as_float(w4[r] << 16), __uint_as_float(w4[r] & 0xFFFF0000u));
+                }
+            }
+        } else {
+            // poll the tagged words of x_l (pairs 2 i, 2 i + 1, i = tid + kThr m)
+            // until every one carries layer l's tag: then every CTA has
+            // finished layer l - 1 (the test hook expects a tag nobody writes)
+            const uint64_t *xw = a.xbuf + (size_t)(l & 1) * H;
+            const uint32_t tag = xch_tag(epoch, l) ^ (a.extra_arrivals && l == 1 ? 1u : 0u);
+            unsigned pend = 0;
+#pragma unroll
+            for (int m = 0; m < kXLoads; ++m)
+                if (2 * (tid + kThr * m) < H) pend |= 1u << m;
+            uint64_t t0 = 0;
+            for (int it = 0; pend; ++it) {
+                uint64_t v[kXLoads][2];
+#pragma unroll
+                for (int m = 0; m < kXLoads; ++m)
+                    if (pend >> m & 1u) ld_tagged2(xw + 2 * (tid + kThr * m), v[m][0], v[m][1]);
+#pragma unroll
+                for (int m = 0; m < kXLoads; ++m)
+                    if ((pend >> m & 1u) && (uint32_t)(v[m][0] >> 32) == tag && (uint32_t)(v[m][1] >> 32) == tag) {
+                        const int i = 2 * (tid + kThr * m);
+                        *reinterpret_cast<float2 *>(xs + xp4(i)) =
+                            make_float2(__uint_as_float((uint32_t)v[m][0] << 16), __uint_as_float((uint32_t)v[m][1] << 16));
+                        pend &= ~(1u << m);
+                    }
+                if (it == 16) t0 = globaltimer_ns();
+                if (pend && it > 16 && (it & 15) == 0) {
+                    if (sh.abort || *(volatile unsigned *)a.ctl != 0u) {
+                        sh.abort = 1;
+                        break;
+                    }
+                    if (deadline_passed(t0, a.timeout_ns)) {
+                        raise_timeout(wc);
+                        break;
+                    }
+                }
+            }
+        }
+        if (__syncthreads_or(sh.abort)) break;
+        stamp(a, l, 4);
         if (warp == 0) {
             // ------------------------------------------ 1a. route, issue copies
             cp_async_wait_all();
@@ -266,37 +352,7 @@ __global__ void __launch_bounds__(kThr, 1) decode1_kernel(const __grid_constant_
             // not wait for it
             if (l + 1 < a.L) fetch_table(a, l + 1, ptab, ltab);
             stamp_dep(a, l, 3, lane == 0, 0.f);
-        } else {
-            // ------------------------------------------ 1b. layer input -> xs
-            const void *xin = l == 0 ? a.x0 : (const void *)(a.xbuf + (size_t)(l & 1) * H);
-            const bool f32 = l == 0 && a.x0_f32;
-            const int per = f32 ? 4 : 8;                // values per 16-byte load
-            const int nld = H / per;
-            uint4 v[kXLoads];
-#pragma unroll
-            for (int q = 0; q < kXLoads; ++q) {
-                const int i = tid - 32 + q * (kThr - 32);
-                if (i < nld) v[q] = __ldcg(static_cast<const uint4 *>(xin) + i);
-            }
-#pragma unroll
-            for (int q = 0; q < kXLoads; ++q) {
-                const int i = tid - 32 + q * (kThr - 32);
-                if (i >= nld) continue;
-                float2 *dst = reinterpret_cast<float2 *>(xs + xp4(i * per));
-                if (f32) {
-                    dst[0] = make_float2(__uint_as_float(v[q].x), __uint_as_float(v[q].y));
-                    dst[1] = make_float2(__uint_as_float(v[q].z), __uint_as_float(v[q].w));
-                } else {
-                    const uint32_t w4[4] = {v[q].x, v[q].y, v[q].z, v[q].w};
-#pragma unroll
-                    for (int r = 0; r < 4; ++r)
-                        dst[r] = make_float2(__uint_as_float(w4[r] << 16), __uint_as_float(w4[r] & 0xFFFF0000u));
-                }
-            }
-            stamp_dep(a, l, 4, tid == 32, __uint_as_float(v[0].x & 0x7F7FFFFFu));
         }
-        if (__syncthreads_or(sh.abort)) break;
-        stamp(a, l, 1);
 
         // ---------------------------------------------- 2. gate/up rows
         // lane: block pb of the row, quarter pq (64 weights, 32 payload bytes).
@@ -325,6 +381,10 @@ __global__ void __launch_bounds__(kThr, 1) decode1_kernel(const __grid_constant_
                 bf16_x_pairs(v, xs_exp, X + 4 * i);
             }
         }
+        // warps 1..7 prepared their activations while warp 0 routed; the
+        // routing's slot table is complete after this
+        if (__syncthreads_or(sh.abort)) break;
+        stamp(a, l, 1);
         bool ok = true;
         for (int j = warp; j < k && ok; j += kW) {
             uint8_t *slot = slots + (size_t)j * a.slot_bytes;
@@ -373,24 +433,17 @@ __global__ void __launch_bounds__(kThr, 1) decode1_kernel(const __grid_constant_
                 const float u = __shfl_down_sync(0xffffffffu, g, 16);
                 const int i = lane >> 2;
                 if (lane < 16 && (lane & 3) == 0 && r0 + i < n_gu)
-                    a.h[(size_t)j * Ip + gu_lo + r0 + i] = silu(g) * u;
+                    st_tagged(a.h + ((size_t)(l & 1) * k + j) * Ip + gu_lo + r0 + i, silu(g) * u, xch_tag(epoch, l));
             }
         }
         if (__syncthreads_or(!ok || sh.abort)) break;
         stamp(a, l, 16);
 
         // ---------------------------------------------- 3. h exchange, down rows
-        unsigned *hcnt = a.ctl + kCtlH + (size_t)l * kCtlHStride;
-        if (tid == 0) {
-            __threadfence();
-            red_release_gpu_add(hcnt, 1u);
-        }
-        // down rows of host slots travel while the counter fills
+        // down rows of host slots travel while other CTAs finish their h rows
         for (int j = warp; j < k; j += kW)
             if (sh.hostmask >> j & 1u)
                 warp_copy_host(slots + (size_t)j * a.slot_bytes + a.down_off, sh.base[j] + sd.src, sd.len);
-        if (tid == 0) wait_counter_ge(wc, hcnt, (unsigned)G);
-        if (__syncthreads_or(sh.abort)) break;
         stamp(a, l, 17);
 
         // this warp's weighted row sums, ysh[warp][ri], summed over its slots.
@@ -402,17 +455,54 @@ __global__ void __launch_bounds__(kThr, 1) decode1_kernel(const __grid_constant_
         for (int j = warp; j < k && ok; j += kW) {
             // h of slot j -> the slot's gate/up part, consumed by now (zeros past
             // I), then the lane's piece and its even/odd sums into registers
-            const float *hj = a.h + (size_t)j * Ip;
+            const uint64_t *hj = a.h + ((size_t)(l & 1) * k + j) * Ip;
             float *hw = reinterpret_cast<float *>(slots + (size_t)j * a.slot_bytes);
             {
-                // every load in flight before the first store (one L2 round trip)
+                // poll the slot's tagged h words (values 4 i .. 4 i + 3 of this
+                // lane's float4 i) until each carries this layer's tag; every
+                // load of a round is in flight before the tags are checked
+                const uint32_t tag = xch_tag(epoch, l);
                 float4 q4[kHLoads];
+                unsigned pend = 0;
 #pragma unroll
                 for (int q = 0; q < kHLoads; ++q) {
                     const int i = lane + 32 * q;
-                    q4[q] = i < Ip / 4 && 4 * i < I ? __ldcg(reinterpret_cast<const float4 *>(hj) + i)
-                                                     : make_float4(0.f, 0.f, 0.f, 0.f);
+                    q4[q] = make_float4(0.f, 0.f, 0.f, 0.f);
+                    if (i < Ip / 4 && 4 * i < I) pend |= 1u << q;
                 }
+                uint64_t t0 = 0;
+                for (int it = 0; __any_sync(0xffffffffu, pend != 0u); ++it) {
+                    uint64_t v[kHLoads][4];
+#pragma unroll
+                    for (int q = 0; q < kHLoads; ++q)
+                        if (pend >> q & 1u) {
+                            const uint64_t *pp = hj + 4 * (lane + 32 * q);
+                            ld_tagged2(pp, v[q][0], v[q][1]);
+                            ld_tagged2(pp + 2, v[q][2], v[q][3]);
+                        }
+#pragma unroll
+                    for (int q = 0; q < kHLoads; ++q)
+                        if ((pend >> q & 1u) && (uint32_t)(v[q][0] >> 32) == tag && (uint32_t)(v[q][1] >> 32) == tag &&
+                            (uint32_t)(v[q][2] >> 32) == tag && (uint32_t)(v[q][3] >> 32) == tag) {
+                            q4[q] = make_float4(__uint_as_float((uint32_t)v[q][0]), __uint_as_float((uint32_t)v[q][1]),
+                                                __uint_as_float((uint32_t)v[q][2]), __uint_as_float((uint32_t)v[q][3]));
+                            pend &= ~(1u << q);
+                        }
+                    if (it == 16) t0 = globaltimer_ns();
+                    if (it > 16 && (it & 15) == 0) {
+                        int stop = sh.abort || *(volatile unsigned *)a.ctl != 0u;
+                        if (!stop && deadline_passed(t0, a.timeout_ns)) {
+                            if (lane == 0) raise_timeout(wc);
+                            stop = 1;
+                        }
+                        if (__any_sync(0xffffffffu, stop)) {
+                            if (lane == 0) sh.abort = 1;
+                            ok = false;
+                            break;
+                        }
+                    }
+                }
+                if (!ok) break;
                 // piece c (64 values) at 68 * c floats: the lanes' pieces start on
                 // distinct bank quads
 #pragma unroll
@@ -484,20 +574,16 @@ __global__ void __launch_bounds__(kThr, 1) decode1_kernel(const __grid_constant_
             const bool last = l == a.L - 1;
             if (a.y) a.y[(size_t)l * H + r] = y;
             if (a.y_bf16 && last) a.y_bf16[r] = float_to_bf16_bits(y);
-            uint16_t *xo = last ? a.x_out : (a.xbuf ? a.xbuf + (size_t)((l + 1) & 1) * H : nullptr);
-            if (xo) xo[r] = float_to_bf16_bits(xs[xp4(r)] + y);
+            const uint16_t xb = float_to_bf16_bits(xs[xp4(r)] + y);
+            if (last) {
+                if (a.x_out) a.x_out[r] = xb;
+            } else if (a.xbuf) {
+                st_tagged(a.xbuf + (size_t)((l + 1) & 1) * H + r, __uint_as_float(xb), xch_tag(epoch, l + 1));
+            }
         }
         stamp(a, l, 20);
-        if (l + 1 < a.L) {
-            __syncthreads();
-            if (tid == 0) {
-                unsigned *bar = a.ctl + kCtlBar + l;
-                __threadfence();
-                red_release_gpu_add(bar, 1u);
-                wait_counter_ge(wc, bar, (unsigned)(G + a.extra_arrivals));
-            }
-            if (__syncthreads_or(sh.abort)) break;
-        }
+        // xs and ysh are read by the combine before the next layer rewrites them
+        if (l + 1 < a.L && __syncthreads_or(sh.abort)) break;
     }
 
     // no copy may still be writing this CTA's shared memory when it exits
@@ -524,6 +610,7 @@ __global__ void __launch_bounds__(kThr, 1) decode1_kernel(const __grid_constant_
     __syncthreads();
     if (sh.last_cta) {
         __threadfence();
+        if (tid == 0) a.ctl[kCtlEpoch] = epoch + 1u;    // the next launch's tags differ
         if (*(volatile unsigned *)a.ctl == 0u) {
             for (int l = tid; l < a.L; l += kThr) {
                 a.ctl[kCtlBar + l] = 0u;
@@ -572,7 +659,7 @@ hfq_status decode1_launch(const hfq4_layer *layers, int L, const float *logits, 
         a.eloc[l] = layers[l].expert_loc;
     }
     a.logits = logits; a.idx_in = idx_in; a.wts_in = wts_in; a.x0 = x0; a.x_out = x_out;
-    a.xbuf = xbuf; a.h = h; a.y = y; a.y_bf16 = y_bf16; a.idx_all = idx_all; a.wts_all = wts_all;
+    a.xbuf = reinterpret_cast<uint64_t *>(xbuf); a.h = reinterpret_cast<uint64_t *>(h); a.y = y; a.y_bf16 = y_bf16; a.idx_all = idx_all; a.wts_all = wts_all;
     a.ctl = ctl; a.timeout_ns = timeout_ns; a.extra_arrivals = extra_arrivals;
     a.timeline = static_cast<unsigned long long *>(option_timeline());
     a.L = L; a.E = E; a.k = k; a.H = H; a.I = I; a.x0_f32 = x0_f32 ? 1 : 0;

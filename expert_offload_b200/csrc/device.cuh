@@ -80,15 +80,19 @@ constexpr size_t kWsHeader = sizeof(WsHeader);   // 256 bytes
 // [64 + l] grid barrier after layer l, [128 + 128 l] CTAs whose h rows of layer
 // l are written.  Zero between launches: the last CTA of a launch clears what
 // it used (a wait that gave up leaves its record until the status is read).
+// After those kCtlWords words, [kCtlEpoch] counts the launches of the
+// one-token kernel on this workspace (its exchange tags); it is never cleared.
 constexpr int kCtlDone = 1, kCtlBar = 64, kCtlH = 128, kCtlHStride = 128;
 constexpr size_t kCtlWords = kCtlH + (size_t)HFQ_MAX_STACK_LAYERS * kCtlHStride;
-constexpr size_t kCtlBytes = (kCtlWords * 4 + 255) / 256 * 256;
+constexpr size_t kCtlEpoch = kCtlWords;
+constexpr size_t kCtlBytes = ((kCtlWords + 1) * 4 + 255) / 256 * 256;
 
 inline cudaError_t launch_check() { return cudaGetLastError(); }
 
 // Persistent decode kernel (stack.cu).
 bool stack_supported(int T, int H, int I, int k, int G);
 size_t stack_ctl_bytes();
+size_t stack_ctl_clear_bytes();      // the leading control words a fresh launch needs at zero
 hfq_status launch_stack(const hfq4_layer *layers, int L, const float *logits, const int32_t *idx_in,
                         const float *wts_in, const void *x0, bool x0_f32, int T, int k,
                         uint16_t *x_out, uint16_t *xbuf, float *h, float *y, uint16_t *y_bf16,

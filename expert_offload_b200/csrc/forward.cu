@@ -152,13 +152,19 @@ __global__ void stack_route_kernel(const float *__restrict__ logits, int T, int 
     }
 }
 
+// h of T tokens x k slots in f32; for one token at least four times that:
+// the one-token kernel exchanges h as 8-byte {value, tag} words in two
+// buffers (layer parity).
 size_t h_bytes(int T, int k, int I)
 {
     size_t nbI = (I + kBlock - 1) / kBlock;
-    return ((size_t)T * k * nbI * kBlock * sizeof(float) + 255) / 256 * 256;
+    return ((size_t)std::max(T, 4) * k * nbI * kBlock * sizeof(float) + 255) / 256 * 256;
 }
 
-size_t act_bytes(int T, int H) { return ((size_t)T * H * 2 + 255) / 256 * 256; }
+// One of the two activation buffers of a decode stack: T x H bf16, and at
+// least H 8-byte words (the one-token kernel's tagged residual stream uses
+// both buffers as [2][H] {bf16 value, tag} words).
+size_t act_bytes(int T, int H) { return (std::max((size_t)T * H * 2, (size_t)H * 8) + 255) / 256 * 256; }
 
 int num_sms_fwd()
 {

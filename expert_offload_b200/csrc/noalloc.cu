@@ -68,7 +68,7 @@ extern "C" hfq_status hfq4_moe_forward_noalloc(const hfq4_layer *layer, const vo
     if (!aligned16(x) || !aligned16(y) || (y_bf16 && !aligned16(y_bf16)))
         return fail(HFQ_ERR_ALIGN, "x, y and y_bf16 must be 16-byte aligned");
     const size_t ip = (size_t)(layer->inter + HFQ4_BLOCK - 1) / HFQ4_BLOCK * HFQ4_BLOCK;
-    const size_t need_h = (size_t)T * k * ip * sizeof(float);
+    const size_t need_h = (size_t)(T < 4 ? 4 : T) * k * ip * sizeof(float);
     if (T < 1 || T > 8 || k > 16 || layer->inter > 1024 || need_h > kNoAllocHBytes ||
         stack_ctl_bytes() > kNoAllocCtlBytes)
         return fail(HFQ_ERR_UNSUPPORTED,
@@ -84,8 +84,10 @@ extern "C" hfq_status hfq4_moe_forward_noalloc(const hfq4_layer *layer, const vo
     if ((st = scratch_address(&scratch))) return st;
     cudaStream_t s = (cudaStream_t)stream;
     // every call shares the array and finds the last call's contents in it:
-    // the control words must start at zero (h is fully rewritten before use)
-    cudaError_t e = cudaMemsetAsync(scratch, 0, stack_ctl_bytes(), s);
+    // the control words must start at zero (h is fully rewritten before use);
+    // the launch epoch after them is kept, so that exchange tags of one call
+    // never match the h words an earlier call left behind
+    cudaError_t e = cudaMemsetAsync(scratch, 0, stack_ctl_clear_bytes(), s);
     if (e != cudaSuccess) return fail(HFQ_ERR_CUDA, "clearing the scratch: %s", cudaGetErrorString(e));
     float *h = reinterpret_cast<float *>(static_cast<char *>(scratch) + kNoAllocCtlBytes);
     st = launch_stack(layer, 1, nullptr, idx, wts, x, x_dtype == HFQ_F32, T, k, nullptr, nullptr, h,

@@ -846,6 +846,8 @@ bool stack_supported(int T, int H, int I, int k, int G)
 
 size_t stack_ctl_bytes() { return kCtlBytes; }
 
+size_t stack_ctl_clear_bytes() { return kCtlWords * 4; }
+
 hfq_status launch_stack(const hfq4_layer *layers, int L, const float *logits, const int32_t *idx_in,
                         const float *wts_in, const void *x0, bool x0_f32, int T, int k,
                         uint16_t *x_out, uint16_t *xbuf, float *h, float *y, uint16_t *y_bf16,
