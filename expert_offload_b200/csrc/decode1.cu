@@ -6,14 +6,15 @@
 // token, a CTA's share of a layer is a fixed pattern: for each routed slot j,
 // rows [c*I/G, (c+1)*I/G) of the expert's gate and up matrices and rows
 // [c*H/G, (c+1)*H/G) of its down matrix (c = this CTA, G = CTAs).  Per layer:
-//   1. warp 0 routes the token (softmax top-k, renormalised; hipfire offload
+//   1. the eight warps route the token (each the top k of an eighth of the
+//      experts, warp 0 merging; softmax top-k, renormalised; hipfire offload
 //      explainer, opening section), reading layer l's logits only after layer
-//      l-1 has finished everywhere, and at once issues the 3k bulk copies
+//      l-1 has finished everywhere, and warp 0 at once issues the 3k bulk copies
 //      (1-D TMA, no multicast), lane j for slot j, into k fixed shared-memory
 //      slots with one mbarrier for gate/up and one for down per slot.  Experts
 //      in host memory are read by the owning warp with 16-byte loads over PCIe
-//      (hipfire offload explainer, "PCIe pass-through").  Warps 1..7 load the
-//      layer input meanwhile.
+//      (hipfire offload explainer, "PCIe pass-through").  Warps 1..7 prepare
+//      their activation registers meanwhile.
 //   2. warp w computes the gate/up rows of slot w (and w + 8) as soon as that
 //      slot has landed: nibbles decoded in registers, warp-shuffle sums,
 //      h = silu(g) * u into an L2-resident buffer as 8-byte {value, tag}
@@ -87,6 +88,8 @@ struct D1Shared {
     int abort;
     int last_cta;
     int armed;                        // layers whose slot barriers were armed
+    uint32_t cand_key[kW * kMaxK];    // routing: each warp's top k of its experts
+    int cand_e[kW * kMaxK];
 };
 
 // Exchange tag of layer l (< 64) in launch `epoch`: never 0 (a fresh
@@ -285,18 +288,18 @@ __global__ void __launch_bounds__(kThr, 1) decode1_kernel(const __grid_constant_
         }
         if (__syncthreads_or(sh.abort)) break;
         stamp(a, l, 4);
+        // ---------------------------------------------- 1b. route (all warps)
+        int re = -1;
+        float rw = 0.0f;
+        if (!a.idx_in) cta_route<kW>(a.logits + (size_t)l * E, E, k, sh.cand_key, sh.cand_e, re, rw);
         if (warp == 0) {
-            // ------------------------------------------ 1a. route, issue copies
+            // ------------------------------------------ 1c. issue copies
             cp_async_wait_all();
             __syncwarp();
             stamp_dep(a, l, 29, lane == 0, 0.f);
-            int e = -1;
-            float w = 0.0f;
-            if (a.idx_in) {
-                if (lane < k) { e = a.idx_in[lane]; w = a.wts_in[lane]; }
-            } else {
-                warp_route(a.logits + (size_t)l * E, E, k, e, w);
-            }
+            int e = re;
+            float w = rw;
+            if (a.idx_in && lane < k) { e = a.idx_in[lane]; w = a.wts_in[lane]; }
             stamp_dep(a, l, 2, lane == 0, w);
             bool bad = lane < k && (unsigned)e >= (unsigned)E;
             const uint8_t *base = nullptr;
