@@ -394,9 +394,9 @@ def run_ours(args, rank, world, local_rank):
     else:
         achieved = bytes_per_step / (mean_launch_ms / 1e3) / 1e9
         # DRAM bytes (read + write) of decode1_kernel from an ncu capture of the
-        # first 10 layers of this workload (133.84 MB read + 5.02 MB written),
+        # first 10 layers of this workload (133.86 MB read + 4.39 MB written),
         # scaled by 4 to the 40-layer launch (the per-layer work is the same)
-        traffic = (133.8368e6 + 5.0196e6) * 4 if (args.workload == "decode" and T == 1
+        traffic = (133.859072e6 + 4.390912e6) * 4 if (args.workload == "decode" and T == 1
                                                  and L == 40 and not args.layers) else None
         out["roofline"] = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak,
                            "unit": "GB/s", "frac": round(achieved / peak, 4), "traffic": traffic,
