@@ -355,6 +355,34 @@ def test_verify_stack_multi_token(eo, verify_model, T):
     assert max(errs) <= TOL, errs
 
 
+def test_one_token_routing_with_ties_across_warps(eo, verify_model):
+    """The one-token kernel routes with all eight warps (each the top k of an
+    eighth of the 512 experts, warp 0 merging the candidates); equal logits
+    must still go to the lower expert index, whichever warps they sit in.
+    Layer 0: every logit equal.  Layer 1: more than k experts spread over all
+    eighths share the largest logit.  Layer 2: logits rounded to a coarse
+    grid (many ties at every rank)."""
+    w, store = verify_model
+    H, I, E, k, L, T = w.hidden, w.inter, w.experts, w.top_k, 3, 1
+    rng = np.random.default_rng(31)
+    logits = np.stack([W.logits(w, l, 900, T) for l in range(L)]).astype(np.float32)
+    logits[0] = 0.25
+    top = np.array([5, 70, 71, 130, 200, 260, 261, 330, 400, 470, 511], np.int64)
+    logits[1, 0, top] = logits[1].max() + 1.0
+    logits[2] = np.round(logits[2] * 2.0) / 2.0
+    x0, _ = W.activations(w, 900, T)
+    x_out, y_all, idx_all, wts_all, _ = _run_stack(eo, store, logits, x0, k, T, H, E, L, I)
+    for l in range(L):
+        ridx, rw = route.route(logits[l], k)
+        np.testing.assert_array_equal(idx_all.cpu().numpy()[l], ridx)
+        np.testing.assert_allclose(wts_all.cpu().numpy()[l], rw, rtol=2e-6, atol=1e-7)
+    np.testing.assert_array_equal(idx_all.cpu().numpy()[0, 0], np.arange(k))
+    np.testing.assert_array_equal(idx_all.cpu().numpy()[1, 0], top[:k])
+    caches = [moe.ExpertCache(OraclePackedLayer(w, l), H, I) for l in range(L)]
+    ys, _ = moe.residual_stack(caches, logits, synth.bf16_bits_to_f32(x0).astype(np.float64), k, route.route)
+    assert max(max_rel_err(y_all.cpu().numpy()[l], ys[l]) for l in range(L)) <= TOL
+
+
 def test_stack_wait_timeout_is_reported_and_recoverable(eo, verify_model):
     """A grid barrier told to wait for a CTA that does not exist runs out after
     the deadline: the status word says HFQ_ERR_TIMEOUT, the kernel winds down
