@@ -248,7 +248,9 @@ hfq_status hfq4_moe_forward_noalloc(const hfq4_layer *layer, const void *x, hfq_
  *     status word, stops doing work, lets its copies in flight land and exits.
  *   HFQ_OPT_TEST_MISSING_ARRIVALS: fault injection for tests; the next
  *     persistent-kernel launch makes its grid barriers wait for this many
- *     CTAs that do not exist, so the wait runs out without any fault.
+ *     CTAs that do not exist (the one-token kernel, which has no grid
+ *     barrier: makes its layer-1 input poll expect a tag nobody writes), so
+ *     the wait runs out without any fault.
  *   HFQ_OPT_TIMELINE_BUFFER: debug; the device address of a u64 buffer of
  *     n_sms * n_layers * 32 words, zero-filled (0 = off).  Persistent-kernel
  *     launches then write %globaltimer stamps (ns), per layer l at word

@@ -384,9 +384,11 @@ def test_one_token_routing_with_ties_across_warps(eo, verify_model):
 
 
 def test_stack_wait_timeout_is_reported_and_recoverable(eo, verify_model):
-    """A grid barrier told to wait for a CTA that does not exist runs out after
-    the deadline: the status word says HFQ_ERR_TIMEOUT, the kernel winds down
-    without faulting, and the next call on the same workspace is correct."""
+    """A cross-CTA wait told to expect what never comes (here, one token: the
+    layer-1 input poll of the one-token kernel waits for a tag nobody writes)
+    runs out after the deadline: the status word says HFQ_ERR_TIMEOUT, the
+    kernel winds down without faulting, and the next call on the same
+    workspace is correct."""
     w, store = verify_model
     H, I, E, k, L, T = w.hidden, w.inter, w.experts, w.top_k, 3, 1
     logits = np.stack([W.logits(w, l, 7, T) for l in range(L)])
