@@ -51,6 +51,23 @@ def test_sizes_match_oracle():
     assert eo.lib().hfq_version() >= 10000
 
 
+@pytest.mark.parametrize("k,H,I,E", [(8, 2048, 512, 256), (8, 2048, 512, 512), (4, 256, 128, 16),
+                                     (16, 1024, 1024, 64)])
+def test_one_token_workspace_holds_the_tagged_exchange_buffers(k, H, I, E):
+    """The one-token kernel exchanges h and the next layer's input as 8-byte
+    {value, tag} words in two buffers (layer parity): the workspace sizes the
+    library reports must hold 2 x k x Ip and 2 x H such words besides the
+    control block (Ip = inter padded to whole 256-weight blocks)."""
+    Ip = -(-I // 256) * 256
+    h_words, x_words = 2 * k * Ip, 2 * H
+    assert eo.hfq4_moe_workspace_bytes(1, k, H, I, E) >= 8 * h_words
+    assert eo.hfq4_stack_workspace_bytes(1, k, H, I, E) >= 8 * (h_words + x_words)
+    # more tokens never need less
+    for T in range(2, 9):
+        assert eo.hfq4_stack_workspace_bytes(T, k, H, I, E) >= eo.hfq4_stack_workspace_bytes(T - 1, k, H, I, E)
+        assert eo.hfq4_stack_workspace_bytes(T, k, H, I, E) % 256 == 0
+
+
 @pytest.mark.parametrize("E,H,I", [(2, 256, 128), (1, 512, 256), (3, 384, 640)])
 def test_host_pack_is_bit_identical_to_oracle(E, H, I):
     rng = np.random.default_rng(E * H + I)
