@@ -72,7 +72,7 @@ struct D1Args {
     unsigned long long *timeline;   // debug: [2][L][kStamps] %globaltimer stamps, or null
     int L, E, k, H, I;
     int x0_f32;
-    int extra_arrivals;       // test hook: grid barriers wait for this many more CTAs
+    int extra_arrivals;       // test hook: nonzero makes the layer-1 input poll expect a tag nobody writes
     // shared-memory layout, bytes; a slot is [gate span][up span][down span]
     int slot_bytes, up_off, down_off;
     int xs_off, ptab_off, ltab_off, ysh_off, sh_off;
