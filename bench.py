@@ -505,7 +505,9 @@ def run_prefill(args):
                       "l2": "256 MB written between timed steps",
                       "gemv_path_ms_per_step": round(ms_gemv, 4),
                       "gemv_path_tokens_per_s": round(T / (ms_gemv / 1e3), 1)},
-           "gpu_launches": 1 + 5, "clocks": clocks,
+           # per step: moe_route (route, group histogram, scan, scatter) and the
+           # tensor-core forward (plan, gather, gate/up, down, combine)
+           "gpu_launches": (4 + 5) * args.steps, "clocks": clocks,
            "roofline": {"bound": "tensor", "achieved": round(achieved, 1), "peak": peak,
                         "unit": "TFLOP/s", "frac": round(achieved / peak, 4), "traffic": None,
                         "flops_per_step": flops,
