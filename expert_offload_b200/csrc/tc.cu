@@ -3,8 +3,11 @@
 //
 // Per expert e with T_e routed (token, slot) pairs (grouped by moe_route):
 //   G = X_e Wg^T, U = X_e Wu^T   (bf16 x bf16 -> f32 in tensor memory)
-//   H_e = bf16(silu(G) * U)
-//   O = H_e Wd^T                  (bf16 x bf16 -> f32), one row per pair
+//   H_e = silu(G) * U, kept as two bf16 parts: hi = bf16(H_e), lo = bf16(H_e - hi)
+//   O = hi Wd^T + lo Wd^T         (bf16 x bf16 -> f32), one row per pair
+// h keeps about 16 significant bits that way: a single bf16 rounding of h
+// would not be unique (a value near a rounding boundary goes either way with
+// f32 errors of the gate/up sums) and would move y by a bf16 step of h.
 //   y[t] = sum_j w_tj * O[pair (t, j)]   (slot order: deterministic)
 // The weights are dequantised from HFQ4 straight into shared memory as bf16,
 // RN_bf16(fmaf(scale, q, zero)), in the canonical K-major no-swizzle layout
@@ -42,11 +45,13 @@ constexpr int kMaxTcCtas = 256;            // grid cap (one CTA per SM); sizes t
 template <bool GU>
 struct TcCfg {
     static constexpr int kRows = GU ? 2 * kM : kM;        // weight rows per item (gate rows, then up rows)
-    static constexpr int kBStages = GU ? 4 : 6;
+    static constexpr int kBStages = 4;
+    static constexpr int kBTiles = GU ? 1 : 2;            // B tiles per stage: x, or h's hi and lo parts
+    static constexpr int kBStageBytes = kBTiles * kTileBytes;
     static constexpr int kABytes = (GU ? 2 : 1) * kTileBytes;
     static constexpr int kRawBytes = kRows * kRawW;
     static constexpr int kBOff = 2 * kABytes;
-    static constexpr int kRawOff = kBOff + kBStages * kTileBytes;
+    static constexpr int kRawOff = kBOff + kBStages * kBStageBytes;
     static constexpr int kSmem = kRawOff + 2 * kRawBytes;
     static constexpr int kDqWords = GU ? 4 : 2;             // nibble words a thread dequantises per stage
     static_assert(kRows * 8 == kDqThr * kDqWords, "one dequantisation task per thread and stage");
@@ -59,7 +64,7 @@ struct TcArgs {
     const void *const *eptr;       // [E] expert base addresses
     const uint8_t *eloc;           // [E] 0 = HBM, 1 = host-mapped, or null
     const int32_t *cnt, *off, *perm;
-    uint16_t *hout;                // gate/up: H_perm out
+    uint16_t *hout;                // gate/up: H_perm out, [pairs][2 I]: hi parts, then lo parts
     float *o;                      // down: O [T*k][H] f32, row q = pair perm[q]
     const int32_t *item_off;       // [E+1] prefix of work items of this phase
     uint8_t *maps;                 // [CTAs][2][128] per-CTA tensor maps of the raw bytes (global)
@@ -288,8 +293,11 @@ __global__ void __launch_bounds__(kTcThr, 1)
             if (kc == 0) p0 = item_of((int)blockIdx.x + it * (int)gridDim.x).p0;
             if (c >= RB && !tc_wait(a, &done_bar[(c - RB) % RB], (uint32_t)((c - RB) / RB) & 1u, abortp)) break;
             if (lane == 0) {
-                mbar_arrive_expect_tx(&fullB[c % RB], (uint32_t)kTileBytes);
-                tma_load_2d(bbuf + (c % RB) * kTileBytes, &bmap, kc * kKC, p0, &fullB[c % RB]);
+                uint8_t *bst = bbuf + (c % RB) * C::kBStageBytes;
+                mbar_arrive_expect_tx(&fullB[c % RB], (uint32_t)C::kBStageBytes);
+                tma_load_2d(bst, &bmap, kc * kKC, p0, &fullB[c % RB]);
+                if (!GU)        // lo part of h, I columns further on
+                    tma_load_2d(bst + kTileBytes, &bmap, a.I + kc * kKC, p0, &fullB[c % RB]);
             }
             nb_issued = c + 1;
             __syncwarp();
@@ -314,14 +322,17 @@ __global__ void __launch_bounds__(kTcThr, 1)
                 // fence orders it before the MMAs' async-proxy reads
                 fence_proxy_async_smem();
                 const uint8_t *A = abuf + (c & 1) * C::kABytes;
-                const uint8_t *B = bbuf + (c % RB) * kTileBytes;
+                const uint8_t *B = bbuf + (c % RB) * C::kBStageBytes;
 #pragma unroll
                 for (int ks = 0; ks < kKC / 16; ++ks) {
                     const uint64_t bd = umma_desc_sw128(B + 32 * ks);
-                    umma_bf16(tmem, umma_desc(A + 2 * ks * kLbo, kLbo, kSbo), bd, idesc, (kc | ks) != 0);
+                    const uint64_t ad = umma_desc(A + 2 * ks * kLbo, kLbo, kSbo);
+                    umma_bf16(tmem, ad, bd, idesc, (kc | ks) != 0);
                     if (GU)
                         umma_bf16(tmem + kN, umma_desc(A + kTileBytes + 2 * ks * kLbo, kLbo, kSbo), bd,
                                   idesc, (kc | ks) != 0);
+                    else        // the same weights against h's lo part
+                        umma_bf16(tmem, ad, umma_desc_sw128(B + kTileBytes + 32 * ks), idesc, true);
                 }
                 umma_commit(&done_bar[c % RB]);
                 tl_stamp(a, GU, c, 6);
@@ -387,9 +398,13 @@ __global__ void __launch_bounds__(kTcThr, 1)
                         const int n = col + jj;
                         if (n >= t.nvalid) break;
                         const int p = t.p0 + n;
-                        if (GU)
-                            a.hout[(size_t)p * a.I + t.r0 + r] = float_to_bf16_bits(silu(g[jj]) * u[jj]);
-                        else
+                        if (GU) {
+                            const float hv = silu(g[jj]) * u[jj];
+                            const uint16_t hi = float_to_bf16_bits(hv);
+                            uint16_t *hrow = a.hout + (size_t)p * 2 * a.I + t.r0 + r;
+                            hrow[0] = hi;
+                            hrow[a.I] = float_to_bf16_bits(hv - bf16_bits_to_float(hi));   // exact difference
+                        } else
                             a.o[(size_t)p * a.H + t.r0 + r] = g[jj];
                     }
                 }
@@ -413,21 +428,32 @@ __global__ void __launch_bounds__(kTcThr, 1)
 
 // Work items per expert: ceil(cnt/kN) token tiles x (rows/kM) row tiles, for
 // the gate/up phase (rows = I) and the down phase (rows = H); exclusive scans.
-__global__ void tc_plan_kernel(const int32_t *__restrict__ cnt, int E, int I, int H,
-                               int32_t *__restrict__ gu_off, int32_t *__restrict__ dn_off)
+// The grouping comes from the caller: unless cnt >= 0, off[0] = 0,
+// off[e + 1] = off[e] + cnt[e] and off[E] = P, the status word gets
+// HFQ_ERR_ARG and both phases get no items (nothing is read or written).
+__global__ void tc_plan_kernel(const int32_t *__restrict__ cnt, const int32_t *__restrict__ off, int E,
+                               int I, int H, int P, int32_t *__restrict__ gu_off, int32_t *__restrict__ dn_off,
+                               unsigned *status)
 {
     __shared__ int s_gu[HFQ_MAX_EXPERTS], s_dn[HFQ_MAX_EXPERTS];
+    __shared__ int s_bad;
+    if (threadIdx.x == 0) s_bad = (off[0] != 0 || off[E] != P);
+    __syncthreads();
     for (int e = threadIdx.x; e < E; e += blockDim.x) {
-        const int tiles = (cnt[e] + kN - 1) / kN;
+        const int c = cnt[e];
+        if (c < 0 || off[e + 1] - off[e] != c) s_bad = 1;
+        const int tiles = c > 0 ? (c + kN - 1) / kN : 0;
         s_gu[e] = tiles * (I / kM);
         s_dn[e] = tiles * (H / kM);
     }
     __syncthreads();
     if (threadIdx.x == 0) {
+        const bool bad = s_bad != 0;
+        if (bad) atomicCAS(status, 0u, (unsigned)HFQ_ERR_ARG);
         int a = 0, b = 0;
         for (int e = 0; e < E; ++e) {
             gu_off[e] = a; dn_off[e] = b;
-            a += s_gu[e]; b += s_dn[e];
+            if (!bad) { a += s_gu[e]; b += s_dn[e]; }
         }
         gu_off[E] = a; dn_off[E] = b;
     }
@@ -436,14 +462,20 @@ __global__ void tc_plan_kernel(const int32_t *__restrict__ cnt, int E, int I, in
 // X_perm[q] = x[token of pair perm[q]] as bf16 (16 bytes per thread step);
 // pos[perm[q]] = q.
 __global__ void tc_gather_kernel(const void *__restrict__ x, int x_f32, const int32_t *__restrict__ perm,
-                                 int P, int k, int H, uint16_t *__restrict__ xp, int32_t *__restrict__ pos)
+                                 int P, int k, int H, uint16_t *__restrict__ xp, int32_t *__restrict__ pos,
+                                 unsigned *status)
 {
     const size_t n8 = (size_t)P * H / 8;
     for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n8;
          i += (size_t)gridDim.x * blockDim.x) {
         const size_t q = i / (H / 8), c = (i - q * (H / 8)) * 8;
-        if (c == 0) pos[perm[q]] = (int32_t)q;
-        const size_t src = (size_t)(perm[q] / k) * H + c;
+        const int pr = perm[q];
+        if ((unsigned)pr >= (unsigned)P) {          // not a pair id: recorded, row left alone
+            if (c == 0) atomicCAS(status, 0u, (unsigned)HFQ_ERR_ARG);
+            continue;
+        }
+        if (c == 0) pos[pr] = (int32_t)q;
+        const size_t src = (size_t)(pr / k) * H + c;
         uint4 v;
         if (x_f32) {
             const float4 a = __ldg(reinterpret_cast<const float4 *>(static_cast<const float *>(x) + src));
@@ -462,18 +494,27 @@ __global__ void tc_gather_kernel(const void *__restrict__ x, int x_f32, const in
 
 // y[t][r] = sum over slots j (in order) of w[t*k + j] * O[pos[t*k + j]][r],
 // four rows per thread step; optional bf16 copy.
+// A pair whose position does not lead back to it (perm was not a permutation
+// of the pairs) is recorded as HFQ_ERR_ARG and left out of the sum.
 __global__ void tc_combine_kernel(const float *__restrict__ o, const int32_t *__restrict__ pos,
-                                  const float *__restrict__ wts, int T, int k, int H, float *__restrict__ y,
-                                  uint16_t *__restrict__ yb)
+                                  const int32_t *__restrict__ perm, const float *__restrict__ wts, int T,
+                                  int k, int H, float *__restrict__ y, uint16_t *__restrict__ yb,
+                                  unsigned *status)
 {
     const size_t n4 = (size_t)T * H / 4;
+    const int P = T * k;
     for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n4;
          i += (size_t)gridDim.x * blockDim.x) {
         const size_t t = i / (H / 4), c = (i - t * (H / 4)) * 4;
         float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
         for (int j = 0; j < k; ++j) {
             const float w = wts[t * k + j];
-            const float4 v = __ldg(reinterpret_cast<const float4 *>(o + (size_t)pos[t * k + j] * H + c));
+            const int q = pos[t * k + j];
+            if ((unsigned)q >= (unsigned)P || perm[q] != (int)(t * k + j)) {
+                if (c == 0) atomicCAS(status, 0u, (unsigned)HFQ_ERR_ARG);
+                continue;
+            }
+            const float4 v = __ldg(reinterpret_cast<const float4 *>(o + (size_t)q * H + c));
             acc.x = fmaf(w, v.x, acc.x);
             acc.y = fmaf(w, v.y, acc.y);
             acc.z = fmaf(w, v.z, acc.z);
@@ -506,8 +547,8 @@ size_t tc_workspace_bytes(int T, int k, int H, int I, int E)
 {
     const size_t P = (size_t)T * k;
     auto r256 = [](size_t b) { return (b + 255) / 256 * 256; };
-    return r256(P * H * 2) + r256(P * I * 2) + 2 * r256((size_t)(E + 1) * 4) + r256(P * H * 4) + r256(P * 4) +
-           r256((size_t)kMaxTcCtas * 256);
+    return r256(P * H * 2) + r256(P * 2 * I * 2) + 2 * r256((size_t)(E + 1) * 4) + r256(P * H * 4) +
+           r256(P * 4) + r256((size_t)kMaxTcCtas * 256);
 }
 
 // Rows of whole HFQ4 blocks must be a multiple of 16 bytes (an even number of
@@ -574,8 +615,8 @@ hfq_status launch_tc(const hfq4_layer &L, const void *x, bool x_f32, int T, int 
     uint8_t *w = static_cast<uint8_t *>(ws);
     uint16_t *xp = reinterpret_cast<uint16_t *>(w);
     w += r256(P * H * 2);
-    uint16_t *hp = reinterpret_cast<uint16_t *>(w);
-    w += r256(P * I * 2);
+    uint16_t *hp = reinterpret_cast<uint16_t *>(w);        // [P][2 I]: hi, lo
+    w += r256(P * 2 * I * 2);
     int32_t *gu_off = reinterpret_cast<int32_t *>(w);
     w += r256((size_t)(E + 1) * 4);
     int32_t *dn_off = reinterpret_cast<int32_t *>(w);
@@ -590,7 +631,7 @@ hfq_status launch_tc(const hfq4_layer &L, const void *x, bool x_f32, int T, int 
     const int rowB_gu = (H + kBlock - 1) / kBlock * kBlockBytes, rowB_dn = (I + kBlock - 1) / kBlock * kBlockBytes;
     const size_t mg = (size_t)I * rowB_gu;
     CUtensorMap xmap, hmap, rmap_gu, rmap_dn;
-    if (!encode_act(&xmap, xp, H, P) || !encode_act(&hmap, hp, I, P) ||
+    if (!encode_act(&xmap, xp, H, P) || !encode_act(&hmap, hp, 2 * I, P) ||
         !encode_raw(&rmap_gu, maps, true, I, rowB_gu, mg) || !encode_raw(&rmap_dn, maps, false, H, rowB_dn, mg))
         return fail(HFQ_ERR_CUDA, "tensor-core path: tensor map encoding failed (H %d, I %d, pairs %zu)", H, I, P);
 
@@ -601,11 +642,11 @@ hfq_status launch_tc(const hfq4_layer &L, const void *x, bool x_f32, int T, int 
         cudaFuncSetAttribute(tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_dn);
         attr = true;
     }
-    tc_plan_kernel<<<1, 512, 0, s>>>(cnt, E, I, H, gu_off, dn_off);
+    tc_plan_kernel<<<1, 512, 0, s>>>(cnt, off, E, I, H, (int)P, gu_off, dn_off, status);
     // pair-ordered bf16 activations (the TMA tiles need contiguous rows)
     const size_t n8 = P * H / 8;
     tc_gather_kernel<<<(unsigned)std::min<size_t>((n8 + 255) / 256, (size_t)tc_sms() * 16), 256, 0, s>>>(
-        x, x_f32 ? 1 : 0, perm, (int)P, k, H, xp, pos);
+        x, x_f32 ? 1 : 0, perm, (int)P, k, H, xp, pos, status);
     TcArgs a;
     a.eptr = L.expert_ptr; a.eloc = L.expert_loc; a.cnt = cnt; a.off = off; a.perm = perm;
     a.maps = maps; a.status = status; a.timeout_ns = timeout_ns; a.E = E; a.H = H; a.I = I; a.k = k;
@@ -616,7 +657,7 @@ hfq_status launch_tc(const hfq4_layer &L, const void *x, bool x_f32, int T, int 
     tc_kernel<false><<<tc_sms(), kTcThr, smem_dn, s>>>(a, hmap, rmap_dn);
     const size_t n4 = (size_t)T * H / 4;
     tc_combine_kernel<<<(unsigned)std::min<size_t>((n4 + 255) / 256, (size_t)tc_sms() * 16), 256, 0, s>>>(
-        ob, pos, wts, T, k, H, y, y_bf16);
+        ob, pos, perm, wts, T, k, H, y, y_bf16, status);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return fail(HFQ_ERR_CUDA, "tensor-core path launch: %s", cudaGetErrorString(e));
     return HFQ_OK;

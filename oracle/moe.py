@@ -10,8 +10,14 @@ with Wg, Wu [I x H] and Wd [H x I] the dequantised HFQ4 matrices (exact
 w = zero + scale*q, see hfq4.py).  No shared expert and no biases.
 
 ``tc=True`` is the numeric model of the bf16 tensor-core path: weights are
-RN_bf16(RN_f32(w)), the activations are already bf16, h is rounded to bf16
-before the down projection, and everything else stays fp64.
+RN_bf16(RN_f32(w)), the activations are already bf16, and everything else
+stays fp64.  h is not rounded: the path carries it into the down projection
+as two bf16 parts (hi = bf16(h), lo = bf16(h - hi), about 16 significant
+bits), whose remaining error is far inside the parity tolerance, whereas a
+single bf16 rounding of h would not be a unique result (values near a
+rounding boundary go either way with the path's f32 errors).  The pages give
+no precision for their tensor-core prefill path (gfx1151 engine README,
+"Windows" section), so this is a stated reading.
 """
 from __future__ import annotations
 
@@ -32,15 +38,18 @@ def round_bf16(a: np.ndarray) -> np.ndarray:
     return r.astype(np.uint32).view(np.float32).astype(np.float64)
 
 
-def expert_ffn(wg: np.ndarray, wu: np.ndarray, wd: np.ndarray, x: np.ndarray,
-               tc: bool = False) -> np.ndarray:
-    """o = Wd (silu(Wg x) * (Wu x)) for x [H] or [T, H] (rows are tokens)."""
+def expert_hidden(wg: np.ndarray, wu: np.ndarray, x: np.ndarray):
+    """(g, u, h) = (Wg x, Wu x, silu(g) * u) for x [H] or [T, H] (rows are
+    tokens), fp64."""
     x = np.asarray(x, dtype=np.float64)
     g = x @ wg.T
     u = x @ wu.T
-    h = silu(g) * u
-    if tc:
-        h = round_bf16(h)
+    return g, u, silu(g) * u
+
+
+def expert_ffn(wg: np.ndarray, wu: np.ndarray, wd: np.ndarray, x: np.ndarray) -> np.ndarray:
+    """o = Wd (silu(Wg x) * (Wu x)) for x [H] or [T, H] (rows are tokens)."""
+    _, _, h = expert_hidden(wg, wu, x)
     return h @ wd.T
 
 
@@ -73,7 +82,7 @@ def moe_layer(experts, hidden: int, inter: int, x: np.ndarray, idx: np.ndarray,
     for t in range(T):
         for j in range(k):
             wg, wu, wd = cache(int(idx[t, j]))
-            y[t] += float(wts[t, j]) * expert_ffn(wg, wu, wd, x[t], tc=cache.tc)
+            y[t] += float(wts[t, j]) * expert_ffn(wg, wu, wd, x[t])
     return y
 
 

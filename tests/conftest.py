@@ -18,3 +18,15 @@ def _built_libs():
     """Build the generator libraries once (host parts are needed on CPU)."""
     import synth
     synth.build()
+
+
+def pytest_terminal_summary(terminalreporter):
+    """Elementwise median and maximum relative errors of every parity
+    comparison that recorded them, beside the normwise metric."""
+    import sys
+    mod = sys.modules.get("tests.gpu_util")
+    lines = mod.report_lines() if mod is not None else []
+    if lines:
+        terminalreporter.section("parity errors (y against the oracle)")
+        for line in lines:
+            terminalreporter.write_line(line)

@@ -12,7 +12,7 @@ import pytest
 import synth
 from oracle import moe, route
 from synth import workloads as W
-from tests.gpu_util import TOL, OraclePackedLayer, device_fill, max_rel_err
+from tests.gpu_util import TOL, OraclePackedLayer, device_fill, oracle_rows, report
 
 pytestmark = pytest.mark.gpu
 torch = pytest.importorskip("torch")
@@ -82,7 +82,7 @@ def test_ragged_persistent_kernels(eo, ragged, T):
     np.testing.assert_array_equal(routed[0].cpu().numpy(), ridx)
     y = _forward(eo, store.layers[0], x, T, k, routed, eo.PATH_AUTO, H, I, E, grouped=False)
     ref = moe.moe_layer(OraclePackedLayer(w, 0), H, I, synth.bf16_bits_to_f32(x).astype(np.float64), ridx, rw)
-    err = max_rel_err(y, ref)
+    err = report(y, ref)
     assert err <= TOL, err
 
 
@@ -96,7 +96,7 @@ def test_ragged_gemv_path(eo, ragged):
     xv = synth.bf16_bits_to_f32(x).astype(np.float64)
     y_gv = _forward(eo, store.layers[0], x, T, k, routed, eo.PATH_GEMV, H, I, E, grouped=False)
     ref_exact = moe.moe_layer(moe.ExpertCache(OraclePackedLayer(w, 0), H, I), H, I, xv, ridx, rw)
-    assert max_rel_err(y_gv, ref_exact) <= TOL
+    assert report(y_gv, ref_exact) <= TOL
 
 
 def test_ragged_shape_without_whole_16_byte_rows_refuses_the_tensor_cores(eo, ragged):
@@ -113,7 +113,7 @@ def test_ragged_shape_without_whole_16_byte_rows_refuses_the_tensor_cores(eo, ra
     ridx, rw = route.route(W.zipf_logits(w, 0, 300, T), k)
     ref = moe.moe_layer(moe.ExpertCache(OraclePackedLayer(w, 0), H, I), H, I,
                         synth.bf16_bits_to_f32(x).astype(np.float64), ridx, rw)
-    assert max_rel_err(y, ref) <= TOL
+    assert report(y, ref) <= TOL
 
 
 @pytest.fixture(scope="module")
@@ -137,6 +137,6 @@ def test_ragged_tensor_core_path(eo, ragged_tc, T):
     ridx, rw = route.route(logits, k)
     xv = synth.bf16_bits_to_f32(x).astype(np.float64)
     y_tc = _forward(eo, store.layers[0], x, T, k, routed, eo.PATH_TC, H, I, E, grouped=True)
-    ref_tc = moe.moe_layer(moe.ExpertCache(OraclePackedLayer(w, 0), H, I, tc=True), H, I, xv, ridx, rw)
-    err = max_rel_err(y_tc, ref_tc)
+    ref_tc = oracle_rows(w, 0, x, ridx, rw, np.arange(T), tc=True, workers=0)
+    err = report(y_tc, ref_tc)
     assert err <= TOL, err

@@ -106,8 +106,8 @@ def test_tc_model_equals_exact_on_representable_values():
     wg, wu, wd = c_exact(0)
     g, u = wg @ x[0], wu @ x[0]
     h = moe.silu(g) * u
-    assert np.array_equal(y1[0], moe.round_bf16(h) @ wd.T)
-    assert np.max(np.abs(y0 - y1)) <= 2**-8 * np.max(np.abs(y0))   # only h's rounding differs
+    assert np.array_equal(y1[0], h @ wd.T)           # h is not rounded in the model
+    assert np.array_equal(y0, y1)
 
 
 def test_round_bf16():
@@ -171,3 +171,25 @@ def test_planted_transposed_down_is_caught():
     a = moe.expert_ffn(wg, wu, wd, x)
     b = moe.expert_ffn(wg, wu, wd.T.copy(), x)
     assert not np.allclose(a, b, rtol=1e-6)
+
+
+def test_grouped_oracle_equals_moe_layer():
+    """The expert-by-expert oracle the full-size GPU checks use
+    (tests/gpu_util.py oracle_rows) gives moe_layer's y, in the exact and the
+    bf16 tensor-core model, for any subset of tokens."""
+    import synth
+    from synth import workloads as W
+    from tests.gpu_util import OraclePackedLayer, oracle_rows
+
+    w = W.WORKLOADS[1]
+    T, k = 8, w.top_k
+    x, _ = W.activations(w, 0, T)
+    x_bits = synth.to_bf16_bits(x.astype(np.float32))
+    xv = synth.bf16_bits_to_f32(x_bits).astype(np.float64)
+    idx, wts = route.route(W.logits(w, 0, 0, T), k)
+    rows = np.array([1, 4, 6])
+    for tc in (False, True):
+        cache = moe.ExpertCache(OraclePackedLayer(w, 0), w.hidden, w.inter, tc=tc)
+        ref = moe.moe_layer(cache, w.hidden, w.inter, xv, idx, wts)
+        y = oracle_rows(w, 0, x_bits, idx, wts, rows, tc=tc, workers=0)
+        np.testing.assert_allclose(y, ref[rows], rtol=1e-12, atol=1e-15)
