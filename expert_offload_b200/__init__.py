@@ -239,7 +239,10 @@ def hfq_set_option(option: int, value: int) -> None:
 
 
 def hfq_workspace_status(workspace, stream=None) -> None:
-    _check(lib().hfq_workspace_status(_ptr(workspace), _nbytes(workspace), _stream(stream)))
+    """Raises HfqError for a device-side error recorded in the workspace; None
+    reads the array of hfq4_moe_forward_noalloc on the current device."""
+    nbytes = 0 if workspace is None else _nbytes(workspace)
+    _check(lib().hfq_workspace_status(_ptr(workspace), nbytes, _stream(stream)))
 
 
 # --------------------------------------------------------- offload plumbing

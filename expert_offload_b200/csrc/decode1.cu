@@ -72,7 +72,8 @@ struct D1Args {
     unsigned long long *timeline;   // debug: [2][L][kStamps] %globaltimer stamps, or null
     int L, E, k, H, I;
     int x0_f32;
-    int extra_arrivals;       // test hook: nonzero makes the layer-1 input poll expect a tag nobody writes
+    int extra_arrivals;       // test hook: nonzero makes the layer-1 input poll (one layer: the h poll)
+                              // expect a tag nobody writes
     // shared-memory layout, bytes; a slot is [gate span][up span][down span]
     int slot_bytes, up_off, down_off;
     int xs_off, ptab_off, ltab_off, ysh_off, sh_off;
@@ -92,15 +93,29 @@ struct D1Shared {
     int cand_e[kW * kMaxK];
 };
 
-// Exchange tag of layer l (< 64) in launch `epoch`: never 0 (a fresh
-// workspace), and as f32 a signalling NaN, which no h value that another
-// kernel leaves in the buffer is.  Every launch rewrites every h word it reads
-// at every layer, so a word holds this launch's previous layer or the last
-// layer of an earlier launch, never a matching tag, whatever the epoch's wrap.
+// Exchange tag of layer l (< 64) in launch `epoch`: never 0 (a fresh or
+// cleared buffer), and as f32 a signalling NaN, which no h value that another
+// kernel leaves in the buffer is.  The epoch keeps 13 bits, so a word last
+// written 8192 launches ago could carry this launch's tag.  That cannot
+// happen while consecutive launches share the exchange layout (k, padded I,
+// H, one layer or several): each launch then rewrites at every layer every
+// word it reads, so an unwritten word holds this launch's layer l - 2 or a
+// layer of one of the two launches before.  When the layout differs from the
+// last launch's (the shape signature below), the first thing a launch does is
+// zero both exchange buffers everywhere, behind one grid-wide counter.
 __device__ __forceinline__ uint32_t xch_tag(uint32_t epoch, int l)
 {
     return 0x7FA00000u | ((epoch & 0x1FFFu) << 7) | (uint32_t)(l + 1);
 }
+
+// Signature of the exchange layout: bit 31 set (0 means none), k, padded I,
+// H and whether x is exchanged (several layers).
+__host__ __device__ __forceinline__ uint32_t xch_signature(int k, int Ip, int H, int L)
+{
+    return 0x80000000u | ((uint32_t)k << 24) | ((uint32_t)(Ip >> 8) << 20) | ((uint32_t)(H >> 3) << 8) |
+           (L > 1 ? 1u : 0u);
+}
+
 
 __device__ __forceinline__ void st_tagged(uint64_t *p, float v, uint32_t tag)
 {
@@ -214,6 +229,8 @@ __global__ void __launch_bounds__(kThr, 1) decode1_kernel(const __grid_constant_
     D1Shared &sh = *reinterpret_cast<D1Shared *>(smem + a.sh_off);
     const WaitCtx wc{a.ctl, a.timeout_ns, &sh.abort};
     const uint32_t epoch = *(volatile const unsigned *)(a.ctl + kCtlEpoch);
+    const uint32_t sig = xch_signature(k, Ip, H, a.L);
+    const bool reset = *(volatile const unsigned *)(a.ctl + kCtlSig) != sig;
 
     if (tid == 0) {
         for (int j = 0; j < kMaxK; ++j) {
@@ -226,9 +243,25 @@ __global__ void __launch_bounds__(kThr, 1) decode1_kernel(const __grid_constant_
     }
     for (int i = H + tid; i < Hp; i += kThr) xs[xp4(i)] = 0.0f;   // padding, never rewritten
     if (warp == 0) fetch_table(a, 0, ptab, ltab);
-    __syncthreads();
+    if (reset) {
+        // another exchange layout ran last on these buffers: zero them (tag 0
+        // matches no launch) and wait until every CTA has done its share
+        const size_t nh = (size_t)2 * k * Ip, nx = a.L > 1 && a.xbuf ? (size_t)2 * H : 0;
+        for (size_t i = (size_t)c * kThr + tid; i < nh + nx; i += (size_t)G * kThr) {
+            if (i < nh) a.h[i] = 0ull;
+            else a.xbuf[i - nh] = 0ull;
+        }
+        __syncthreads();
+        if (tid == 0) {
+            __threadfence();
+            atomicAdd(a.ctl + kCtlClear, 1u);
+            if (!wait_counter_ge(wc, a.ctl + kCtlClear, (unsigned)G)) sh.abort = 1;
+        }
+    }
+    // a reset that did not complete leaves the layers undone (nothing armed)
+    const int n_layers = __syncthreads_or(sh.abort) ? 0 : a.L;
 
-    for (int l = 0; l < a.L; ++l) {
+    for (int l = 0; l < n_layers; ++l) {
         stamp(a, l, 0);
         const uint32_t par = l & 1;          // parity of this layer's slot-barrier phases
         // ---------------------------------------------- 1a. layer input -> xs
@@ -463,8 +496,9 @@ __global__ void __launch_bounds__(kThr, 1) decode1_kernel(const __grid_constant_
             {
                 // poll the slot's tagged h words (values 4 i .. 4 i + 3 of this
                 // lane's float4 i) until each carries this layer's tag; every
-                // load of a round is in flight before the tags are checked
-                const uint32_t tag = xch_tag(epoch, l);
+                // load of a round is in flight before the tags are checked (the
+                // test hook of a one-layer launch expects a tag nobody writes)
+                const uint32_t tag = xch_tag(epoch, l) ^ (a.extra_arrivals && a.L == 1 ? 1u : 0u);
                 float4 q4[kHLoads];
                 unsigned pend = 0;
 #pragma unroll
@@ -613,7 +647,10 @@ __global__ void __launch_bounds__(kThr, 1) decode1_kernel(const __grid_constant_
     __syncthreads();
     if (sh.last_cta) {
         __threadfence();
-        if (tid == 0) a.ctl[kCtlEpoch] = epoch + 1u;    // the next launch's tags differ
+        if (tid == 0) {
+            a.ctl[kCtlEpoch] = epoch + 1u;    // the next launch's tags differ
+            a.ctl[kCtlSig] = sig;             // and it knows this launch's layout
+        }
         if (*(volatile unsigned *)a.ctl == 0u) {
             for (int l = tid; l < a.L; l += kThr) {
                 a.ctl[kCtlBar + l] = 0u;
@@ -622,6 +659,7 @@ __global__ void __launch_bounds__(kThr, 1) decode1_kernel(const __grid_constant_
             __syncthreads();
             if (tid == 0) {
                 __threadfence();
+                a.ctl[kCtlClear] = 0u;
                 a.ctl[kCtlDone] = 0u;
             }
         }

@@ -80,12 +80,17 @@ constexpr size_t kWsHeader = sizeof(WsHeader);   // 256 bytes
 // [64 + l] grid barrier after layer l, [128 + 128 l] CTAs whose h rows of layer
 // l are written.  Zero between launches: the last CTA of a launch clears what
 // it used (a wait that gave up leaves its record until the status is read).
-// After those kCtlWords words, [kCtlEpoch] counts the launches of the
-// one-token kernel on this workspace (its exchange tags); it is never cleared.
-constexpr int kCtlDone = 1, kCtlBar = 64, kCtlH = 128, kCtlHStride = 128;
+// [2] counts the CTAs of a one-token launch that have cleared its exchange
+// buffers (only when the shape signature below changed).  After those
+// kCtlWords words, [kCtlEpoch] counts the launches of the one-token kernel on
+// this workspace (its exchange tags) and [kCtlSig] holds the shape signature
+// of the last one (0 = none yet); neither is cleared between launches, and
+// both are cleared with the control block after a device-side error.
+constexpr int kCtlDone = 1, kCtlClear = 2, kCtlBar = 64, kCtlH = 128, kCtlHStride = 128;
 constexpr size_t kCtlWords = kCtlH + (size_t)HFQ_MAX_STACK_LAYERS * kCtlHStride;
 constexpr size_t kCtlEpoch = kCtlWords;
-constexpr size_t kCtlBytes = ((kCtlWords + 1) * 4 + 255) / 256 * 256;
+constexpr size_t kCtlSig = kCtlWords + 1;
+constexpr size_t kCtlBytes = ((kCtlWords + 2) * 4 + 255) / 256 * 256;
 
 inline cudaError_t launch_check() { return cudaGetLastError(); }
 
@@ -124,6 +129,10 @@ hfq_status launch_tc(const hfq4_layer &L, const void *x, bool x_f32, int T, int 
                      const int32_t *off, const int32_t *perm, const float *wts, float *y,
                      uint16_t *y_bf16, void *ws, unsigned *status, long long timeout_ns,
                      cudaStream_t s);
+
+// Status word of the allocation-free forward's array on the current device
+// (noalloc.cu); hfq_workspace_status(NULL, 0, stream) returns it.
+hfq_status noalloc_status(cudaStream_t s);
 
 // Library options (hfq_set_option).
 long long option_wait_timeout_ns();

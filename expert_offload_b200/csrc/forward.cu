@@ -46,18 +46,31 @@ __device__ __forceinline__ float row_dot(const uint8_t *__restrict__ row, int nb
     return warp_sum(acc);
 }
 
+// An expert id from the caller outside [0, E): recorded as HFQ_ERR_ARG in the
+// status word (read by hfq_workspace_status); the pair is skipped, so no
+// address is formed from it.
+__device__ __forceinline__ bool bad_expert(int e, int E, unsigned *status)
+{
+    if ((unsigned)e < (unsigned)E) return false;
+    if (status) atomicCAS(status, 0u, (unsigned)HFQ_ERR_ARG);
+    return true;
+}
+
 // Gate/up: CTA (pair p = t*k + j, row chunk).  h[p][r] = silu(g_r) * u_r.
 __global__ void __launch_bounds__(kThreads)
 gateup_kernel(const void *const *__restrict__ eptr, const void *__restrict__ x, int x_dtype,
-              const int32_t *__restrict__ idx, int k, int H, int I, float *__restrict__ h)
+              const int32_t *__restrict__ idx, int k, int E, int H, int I, float *__restrict__ h,
+              unsigned *status)
 {
     extern __shared__ float xs[];               // [nbH * 256]
     const int p = blockIdx.x, t = p / k;
+    const int e = idx[p];
+    if (bad_expert(e, E, threadIdx.x == 0 ? status : nullptr)) return;
     const int nbH = (H + kBlock - 1) / kBlock;
     for (int i = threadIdx.x; i < nbH * kBlock; i += kThreads)
         xs[i] = i < H ? load_act(x, x_dtype, (size_t)t * H + i) : 0.0f;
     __syncthreads();
-    const uint8_t *base = static_cast<const uint8_t *>(eptr[idx[p]]);
+    const uint8_t *base = static_cast<const uint8_t *>(eptr[e]);
     const size_t row_bytes = (size_t)nbH * kBlockBytes;
     const uint8_t *gate = base, *up = base + (size_t)I * row_bytes;
     const int warp = threadIdx.x >> 5;
@@ -75,12 +88,16 @@ gateup_kernel(const void *const *__restrict__ eptr, const void *__restrict__ x, 
 // With x_res != null also writes x_next[t][r] = bf16(x_res[t][r] + y[t][r]).
 __global__ void __launch_bounds__(kThreads)
 down_kernel(const void *const *__restrict__ eptr, const float *__restrict__ h,
-            const int32_t *__restrict__ idx, const float *__restrict__ wts, int k, int H, int I,
+            const int32_t *__restrict__ idx, const float *__restrict__ wts, int k, int E, int H, int I,
             float *__restrict__ y, uint16_t *__restrict__ y_bf16,
-            const uint16_t *__restrict__ x_res, uint16_t *__restrict__ x_next)
+            const uint16_t *__restrict__ x_res, uint16_t *__restrict__ x_next, unsigned *status)
 {
     extern __shared__ float hs[];               // [k][nbI * 256]
     const int t = blockIdx.x;
+    // a token with an invalid expert id writes nothing (its gate/up pairs were
+    // skipped too); the status word says why
+    for (int j = 0; j < k; ++j)
+        if (bad_expert(idx[(size_t)t * k + j], E, threadIdx.x == 0 ? status : nullptr)) return;
     const int nbI = (I + kBlock - 1) / kBlock, hl = nbI * kBlock;
     for (int i = threadIdx.x; i < k * hl; i += kThreads) {
         int j = i / hl, c = i - j * hl;
@@ -188,7 +205,7 @@ hfq_status check_ws(void *ws, size_t ws_bytes, size_t need)
 
 hfq_status launch_layer(const hfq4_layer &L, const void *x, int x_dtype, int T, const int32_t *idx,
                         const float *wts, int k, float *y, void *y_bf16, float *h,
-                        const uint16_t *x_res, uint16_t *x_next, cudaStream_t s)
+                        const uint16_t *x_res, uint16_t *x_next, unsigned *status, cudaStream_t s)
 {
     const int H = L.hidden, I = L.inter;
     const int nbH = (H + kBlock - 1) / kBlock, nbI = (I + kBlock - 1) / kBlock;
@@ -204,10 +221,11 @@ hfq_status launch_layer(const hfq4_layer &L, const void *x, int x_dtype, int T, 
     }
     dim3 g1(T * k, (I + kRowsPerCta - 1) / kRowsPerCta);
     gateup_kernel<<<g1, kThreads, nbH * kBlock * sizeof(float), s>>>(
-        L.expert_ptr, x, x_dtype, idx, k, H, I, h);
+        L.expert_ptr, x, x_dtype, idx, k, L.n_experts, H, I, h, status);
     dim3 g2(T, (H + kRowsPerCta - 1) / kRowsPerCta);
     down_kernel<<<g2, kThreads, smem_down, s>>>(
-        L.expert_ptr, h, idx, wts, k, H, I, y, static_cast<uint16_t *>(y_bf16), x_res, x_next);
+        L.expert_ptr, h, idx, wts, k, L.n_experts, H, I, y, static_cast<uint16_t *>(y_bf16), x_res, x_next,
+        status);
     cudaError_t err = cudaGetLastError();
     if (err != cudaSuccess) return fail(HFQ_ERR_CUDA, "forward launch: %s", cudaGetErrorString(err));
     return HFQ_OK;
@@ -309,7 +327,8 @@ hfq_status hfq4_moe_forward(const hfq4_layer *layer, const void *x, hfq_dtype x_
                           static_cast<unsigned *>(workspace), option_wait_timeout_ns(),
                           option_take_extra_arrivals(), s);
     } else {
-        st = launch_layer(*layer, x, x_dtype, T, idx, wts, k, y, y_bf16, h, nullptr, nullptr, s);
+        st = launch_layer(*layer, x, x_dtype, T, idx, wts, k, y, y_bf16, h, nullptr, nullptr,
+                          static_cast<unsigned *>(workspace), s);
     }
     return st ? st : ok();
 }
@@ -376,7 +395,8 @@ hfq_status hfq4_moe_decode_stack(const hfq4_layer *layers, int n_layers, const f
                                                 idx_all ? idx_all + (size_t)l * T * k : nullptr,
                                                 wts_all ? wts_all + (size_t)l * T * k : nullptr);
         float *y = y_all ? y_all + (size_t)l * T * H : nullptr;
-        st = launch_layer(layers[l], cur, HFQ_BF16, T, idx, wts, k, y, nullptr, h, cur, next, s);
+        st = launch_layer(layers[l], cur, HFQ_BF16, T, idx, wts, k, y, nullptr, h, cur, next,
+                          static_cast<unsigned *>(workspace), s);
         if (st) return st;
         cur = next;
     }
@@ -385,6 +405,7 @@ hfq_status hfq4_moe_decode_stack(const hfq4_layer *layers, int n_layers, const f
 
 hfq_status hfq_workspace_status(void *workspace, size_t ws_bytes, void *stream)
 {
+    if (!workspace && ws_bytes == 0) return noalloc_status((cudaStream_t)stream);
     if (!workspace || ws_bytes < kWsHeader) return fail(HFQ_ERR_ARG, "no workspace");
     unsigned int word = 0;
     cudaStream_t s = (cudaStream_t)stream;
@@ -396,7 +417,10 @@ hfq_status hfq_workspace_status(void *workspace, size_t ws_bytes, void *stream)
         size_t n = ws_bytes < stack_ctl_bytes() ? ws_bytes : stack_ctl_bytes();
         cudaMemsetAsync(workspace, 0, n, s);
         cudaStreamSynchronize(s);
-        return fail((hfq_status)(int)word, "a device-side wait ran out (status %d)", (int)word);
+        const int st = (int)word;
+        if (st == HFQ_ERR_ARG)
+            return fail(HFQ_ERR_ARG, "a kernel found an invalid expert id or grouping (status %d)", st);
+        return fail((hfq_status)st, "a device-side wait ran out (status %d)", st);
     }
     return ok();
 }

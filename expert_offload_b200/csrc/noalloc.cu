@@ -51,6 +51,35 @@ hfq_status scratch_address(void **out)
 }
 
 }  // namespace
+
+// hfq_workspace_status(NULL, 0, stream): the status word of this device's
+// array.  HFQ_OK when no call has run on the device yet.  After an error the
+// array's control block is cleared, as a workspace's would be.
+hfq_status noalloc_status(cudaStream_t s)
+{
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return fail(HFQ_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
+    void *scratch = nullptr;
+    {
+        std::lock_guard<std::mutex> g(g_mu);
+        if (dev >= 0 && dev < kMaxDevices) scratch = g_scratch_ptr[dev];
+    }
+    if (!scratch) return ok();
+    unsigned word = 0;
+    e = cudaMemcpyAsync(&word, scratch, sizeof word, cudaMemcpyDeviceToHost, s);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+    if (e != cudaSuccess) return fail(HFQ_ERR_CUDA, "status read: %s", cudaGetErrorString(e));
+    if (word == 0) return ok();
+    e = cudaMemsetAsync(scratch, 0, stack_ctl_bytes(), s);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+    if (e != cudaSuccess) return fail(HFQ_ERR_CUDA, "clearing the scratch: %s", cudaGetErrorString(e));
+    const int st = (int)word;
+    if (st == HFQ_ERR_ARG)
+        return fail(HFQ_ERR_ARG, "the allocation-free forward found an invalid expert id (status %d)", st);
+    return fail((hfq_status)st, "a device-side wait of the allocation-free forward ran out (status %d)", st);
+}
+
 }  // namespace hfq
 
 using namespace hfq;
@@ -69,25 +98,28 @@ extern "C" hfq_status hfq4_moe_forward_noalloc(const hfq4_layer *layer, const vo
         return fail(HFQ_ERR_ALIGN, "x, y and y_bf16 must be 16-byte aligned");
     const size_t ip = (size_t)(layer->inter + HFQ4_BLOCK - 1) / HFQ4_BLOCK * HFQ4_BLOCK;
     const size_t need_h = (size_t)(T < 4 ? 4 : T) * k * ip * sizeof(float);
-    if (T < 1 || T > 8 || k > 16 || layer->inter > 1024 || need_h > kNoAllocHBytes ||
-        stack_ctl_bytes() > kNoAllocCtlBytes)
+    if (T < 1 || T > 8 || k > 16 || layer->inter > 1024 || layer->hidden > 2048 ||
+        need_h > kNoAllocHBytes || stack_ctl_bytes() > kNoAllocCtlBytes)
         return fail(HFQ_ERR_UNSUPPORTED,
-                    "hfq4_moe_forward_noalloc takes T <= 8, k <= 16, inter <= 1024 (its fixed "
-                    "scratch is %zu bytes); got T=%d k=%d inter=%d", kNoAllocBytes, T, k,
-                    layer->inter);
+                    "hfq4_moe_forward_noalloc takes T <= 8, k <= 16, inter <= 1024, hidden <= 2048 "
+                    "(its fixed scratch is %zu bytes); got T=%d k=%d inter=%d hidden=%d", kNoAllocBytes,
+                    T, k, layer->inter, layer->hidden);
     int sms = 0, dev = 0;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return fail(HFQ_ERR_CUDA, "device query: %s", cudaGetErrorString(e));
     if (!stack_supported(T, layer->hidden, layer->inter, k, sms))
-        return fail(HFQ_ERR_UNSUPPORTED, "shape not supported by the persistent kernel");
+        return fail(HFQ_ERR_UNSUPPORTED, "hfq4_moe_forward_noalloc: shape (T=%d k=%d hidden=%d inter=%d) "
+                    "not supported by the persistent kernel", T, k, layer->hidden, layer->inter);
     void *scratch = nullptr;
     if ((st = scratch_address(&scratch))) return st;
     cudaStream_t s = (cudaStream_t)stream;
     // every call shares the array and finds the last call's contents in it:
-    // the control words must start at zero (h is fully rewritten before use);
-    // the launch epoch after them is kept, so that exchange tags of one call
-    // never match the h words an earlier call left behind
-    cudaError_t e = cudaMemsetAsync(scratch, 0, stack_ctl_clear_bytes(), s);
+    // the control words (the status word among them) must start at zero; the
+    // launch epoch and layout signature after them are kept, so that the
+    // one-token kernel's exchange tags never match h words an earlier call
+    // left behind (a call with another k or inter clears h first)
+    e = cudaMemsetAsync(scratch, 0, stack_ctl_clear_bytes(), s);
     if (e != cudaSuccess) return fail(HFQ_ERR_CUDA, "clearing the scratch: %s", cudaGetErrorString(e));
     float *h = reinterpret_cast<float *>(static_cast<char *>(scratch) + kNoAllocCtlBytes);
     st = launch_stack(layer, 1, nullptr, idx, wts, x, x_dtype == HFQ_F32, T, k, nullptr, nullptr, h,

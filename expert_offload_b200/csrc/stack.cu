@@ -375,7 +375,14 @@ __global__ void __launch_bounds__(kThr, 1) stack_kernel(const __grid_constant__ 
             const int t = warp - route_w0;
             if (a.idx_in) {
                 for (int j = lane; j < a.k; j += 32) {
-                    sh.sel[t][j] = a.idx_in[t * a.k + j];
+                    int e = a.idx_in[t * a.k + j];
+                    if ((unsigned)e >= (unsigned)a.E) {
+                        // a caller's id outside [0, E): recorded; expert 0 stands
+                        // in so that every table index stays in range
+                        atomicCAS(a.ctl, 0u, (unsigned)HFQ_ERR_ARG);
+                        e = 0;
+                    }
+                    sh.sel[t][j] = e;
                     sh.wsel[t][j] = a.wts_in[t * a.k + j];
                 }
             } else {

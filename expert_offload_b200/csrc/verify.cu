@@ -275,7 +275,14 @@ __global__ void __launch_bounds__(kThr, 1) verify_kernel(const __grid_constant__
         if (warp < T) {
             if (a.idx_in) {
                 for (int j = lane; j < k; j += 32) {
-                    sh.sel[warp][j] = a.idx_in[warp * k + j];
+                    int e = a.idx_in[warp * k + j];
+                    if ((unsigned)e >= (unsigned)a.E) {
+                        // a caller's id outside [0, E): recorded; expert 0 stands
+                        // in so that every table index stays in range
+                        atomicCAS(a.ctl, 0u, (unsigned)HFQ_ERR_ARG);
+                        e = 0;
+                    }
+                    sh.sel[warp][j] = e;
                     sh.wsel[warp][j] = a.wts_in[warp * k + j];
                 }
             } else {

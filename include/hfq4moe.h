@@ -176,7 +176,8 @@ typedef struct {
  *           TC forces the tensor-core path (HFQ_ERR_UNSUPPORTED for other
  *           shapes) [WMMA]: weights dequantised to RN_bf16(fmaf(scale, q, zero)),
  *           x rounded to bf16 (exact for bf16 input), f32 accumulation, h
- *           rounded to bf16 before the down projection, each pair's down
+ *           carried into the down projection as two bf16 parts (hi and the
+ *           bf16 rounding of h - hi, about 16 significant bits), each pair's down
  *           output kept in f32 and y summed over the k slots in slot order
  *           (deterministic).
  *   y:      f32 [T][H] out.  y_bf16: optional bf16 [T][H] out (NULL = none).
@@ -233,8 +234,15 @@ hfq_status hfq4_moe_decode_stack(const hfq4_layer *layers, int n_layers, const f
  *   The first call on a device looks up the array's device address for that
  *   device (with that device current); make that first call before any stream
  *   capture.  Each call clears the array's control words on `stream` before
- *   launching.  All calls share the one array, so calls that overlap on the
- *   GPU (different streams without ordering) race; order them on one stream.
+ *   launching, the status word among them.  All calls share the one array, so
+ *   calls that overlap on the GPU (different streams without ordering) race;
+ *   order them on one stream.  Calls may change k, T and the layer's shape
+ *   from one to the next: a one-token call whose exchange layout (k, inter,
+ *   hidden) differs from the last one's clears the array's h part first.
+ *   Device-side conditions (a bounded wait that ran out, an expert id outside
+ *   [0, n_experts)) go to the array's status word: read it with
+ *   hfq_workspace_status(NULL, 0, stream) after the call and before the next
+ *   one, which clears it.
  */
 hfq_status hfq4_moe_forward_noalloc(const hfq4_layer *layer, const void *x, hfq_dtype x_dtype,
                                     int T, const int32_t *idx, const float *wts, int k, float *y,
@@ -249,8 +257,8 @@ hfq_status hfq4_moe_forward_noalloc(const hfq4_layer *layer, const void *x, hfq_
  *   HFQ_OPT_TEST_MISSING_ARRIVALS: fault injection for tests; the next
  *     persistent-kernel launch makes its grid barriers wait for this many
  *     CTAs that do not exist (the one-token kernel, which has no grid
- *     barrier: makes its layer-1 input poll expect a tag nobody writes), so
- *     the wait runs out without any fault.
+ *     barrier: makes its layer-1 input poll, or with one layer its h poll,
+ *     expect a tag nobody writes), so the wait runs out without any fault.
  *   HFQ_OPT_TIMELINE_BUFFER: debug; the device address of a u64 buffer of
  *     n_sms * n_layers * 32 words, zero-filled (0 = off).  Persistent-kernel
  *     launches then write %globaltimer stamps (ns), per layer l at word
@@ -271,10 +279,15 @@ hfq_status hfq4_moe_forward_noalloc(const hfq4_layer *layer, const void *x, hfq_
 hfq_status hfq_set_option(int option, long long value);
 
 /*
- * Device status word of a workspace (synchronises `stream`): HFQ_OK, or
- * HFQ_ERR_TIMEOUT if a bounded device-side wait of a previous call ran out.
- * After a timeout the word and the workspace's control block are cleared.
- * A new workspace must be zero-filled before its first use.
+ * Device status word of a workspace (synchronises `stream`): HFQ_OK,
+ * HFQ_ERR_TIMEOUT if a bounded device-side wait of a previous call ran out, or
+ * HFQ_ERR_ARG if a kernel met an expert id outside [0, n_experts) or (tensor-
+ * core path) a grouping whose cnt/off/perm do not describe the T*k pairs; the
+ * work of such a pair is skipped, its output left unwritten.  After an error
+ * the word and the workspace's control block are cleared.  A new workspace
+ * must be zero-filled before its first use.  workspace = NULL with
+ * ws_bytes = 0 reads the status word of hfq4_moe_forward_noalloc's array on
+ * the current device (HFQ_OK when no such call has run there).
  */
 hfq_status hfq_workspace_status(void *workspace, size_t ws_bytes, void *stream);
 

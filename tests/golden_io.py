@@ -39,3 +39,16 @@ def load_hfq4_cases(name="hfq4_handpacked.txt"):
         c["bytes"] = np.array(c["bytes"], dtype=np.uint8)
         c["expect"] = np.array(c["expect"], dtype=np.float64).reshape(c["rows"], c["cols"])
     return cases
+
+
+def load_placement_cases(name="placement_auto.txt"):
+    """Rows of the hand-worked placement fixture as dicts."""
+    keys = ["name", "resident", "hot", "budget", "ok", "N", "hbm", "host", "deficit"]
+    out = []
+    for line in open(os.path.join(GOLDEN, name)):
+        if line.startswith("case "):
+            f = line.split()[1:]
+            d = dict(zip(keys, [f[0]] + [int(v) for v in f[1:]]))
+            d["ok"] = bool(d["ok"])
+            out.append(d)
+    return out

@@ -137,3 +137,35 @@ def test_argument_errors_are_caught_before_launch():
     assert "16-byte" in eo.last_error()
     assert lib.hfq4_dequant(1028, 1, 256, 1024, None) == -2
     assert lib.hfq_host_arena_destroy(12345) == -1
+
+
+def test_placement_hand_worked_cases():
+    """The library's placement on the hand-worked cases of
+    tests/golden/placement_auto.txt (40 layers x 256 experts of 1,671,168 bytes)."""
+    from tests.golden_io import load_placement_cases
+    L, E, eb = 40, 256, 1_671_168
+    counts = np.tile(np.arange(E, dtype=np.uint32), (L, 1))
+    for c in load_placement_cases():
+        if c["ok"]:
+            loc, slot, hn, hs = eo.hfq_placement_build(counts, eb, c["resident"], c["hot"], c["budget"])
+            assert (hn, hs) == (c["hbm"], c["host"]), c["name"]
+            assert int((loc[:, :] == 0).all(axis=1).sum()) == c["N"], c["name"]
+        else:
+            with pytest.raises(eo.HfqError) as e:
+                eo.hfq_placement_build(counts, eb, c["resident"], c["hot"], c["budget"])
+            assert e.value.status == -4, c["name"]
+            assert f"deficit {c['deficit']}" in e.value.message, c["name"]
+            assert (e.value.hbm_needed, e.value.host_needed) == (c["hbm"], c["host"]), c["name"]
+
+
+def test_host_arena_refuses_an_impossible_size():
+    """Allocation failure of the pinned expert arena is reported as
+    HFQ_ERR_ALLOC with the byte count, for both page-size choices (no GPU
+    needed: the request fails before any device is involved or at the
+    registration)."""
+    huge = 1 << 60
+    for flags in (0, eo.ARENA_HUGEPAGE):
+        with pytest.raises(eo.HfqError) as e:
+            eo.hfq_host_arena_create(huge, flags)
+        assert e.value.status == -7
+        assert str(huge) in e.value.message

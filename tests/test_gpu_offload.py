@@ -8,7 +8,7 @@ import pytest
 import synth
 from oracle import moe, placement, route
 from synth import workloads as W
-from tests.gpu_util import TOL, OraclePackedLayer, device_fill, max_rel_err
+from tests.gpu_util import TOL, OraclePackedLayer, device_fill, report
 
 pytestmark = pytest.mark.gpu
 torch = pytest.importorskip("torch")
@@ -65,7 +65,7 @@ def test_offloaded_stack_matches_oracle(eo, offload_model, T):
     caches = [moe.ExpertCache(OraclePackedLayer(w, l), H, I) for l in range(L)]
     ys, _ = moe.residual_stack(caches, logits, synth.bf16_bits_to_f32(x0).astype(np.float64), k,
                                route.route)
-    errs = [max_rel_err(y_all.cpu().numpy()[l], ys[l]) for l in range(L)]
+    errs = [report(y_all.cpu().numpy()[l], ys[l]) for l in range(L)]
     assert max(errs) <= TOL, errs
 
 

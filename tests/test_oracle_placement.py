@@ -59,3 +59,24 @@ def test_slots_are_dense_per_location():
     for where in (0, 1):
         s = sorted(p.slot[p.loc == where].tolist())
         assert s == list(range(len(s)))
+
+
+def test_hand_worked_auto_placement_of_the_explainers_40_layer_model():
+    """tests/golden/placement_auto.txt: the 40-layer, 408 MiB-per-layer model
+    of the explainer's measurements, worked out by hand (auto with and without
+    hot sets, and both refusals)."""
+    from tests.golden_io import load_placement_cases
+    L, E, eb = 40, 256, 1_671_168
+    counts = np.tile(np.arange(E, dtype=np.uint32), (L, 1))      # c[l][e] = e
+    cases = load_placement_cases()
+    assert len(cases) == 4
+    for c in cases:
+        p = P.place(counts, eb, c["resident"], c["hot"], c["budget"])
+        assert p.ok == c["ok"], c["name"]
+        assert p.resident_layers == c["N"], c["name"]
+        assert (p.hbm_needed, p.host_needed, p.deficit) == (c["hbm"], c["host"], c["deficit"]), c["name"]
+        if c["ok"]:
+            N, h = c["N"], c["hot"]
+            assert np.all(p.loc[:N] == P.HBM)
+            for l in range(N, L):
+                assert np.nonzero(p.loc[l] == P.HBM)[0].tolist() == list(range(E - h, E))
