@@ -33,29 +33,35 @@ constexpr int kBWarp = kDqW + 1;           // TMA loads of the activation tiles
 constexpr int kRawWarp = kDqW + 2;         // TMA loads of the raw HFQ4 bytes
 constexpr int kTcThr = (kDqW + 3) * 32;
 constexpr int kTileBytes = kM * kKC * 2;   // one 128 x kKC bf16 operand tile (16 KB)
-constexpr uint32_t kLbo = (kM / 8) * 128;  // no-swizzle A tiles: bytes between 8-element K chunks
-constexpr uint32_t kSbo = 128;             // no-swizzle A tiles: bytes between 8-row groups
 constexpr int kRawW = 144;                 // staged bytes per weight row and HFQ4 block (16-byte window)
-constexpr uint32_t kTmemCols = 256;
 constexpr int kMaxTcCtas = 256;            // grid cap (one CTA per SM); sizes the tensor-map slots
 
-// Shared memory of one phase: two dequantised A buffers (gate [+ up]), a ring
-// of activation B tiles (TMA, 128-byte swizzle) and two raw buffers, each the
-// 144-byte window around one HFQ4 block of every weight row of the item.
+// One phase's buffers.  Shared memory: a ring of activation B tiles (TMA,
+// 128-byte swizzle) and two raw buffers, each the 144-byte window around one
+// HFQ4 block of every weight row of the item.  Tensor memory: the f32
+// accumulators (gate [+ up]: kN columns each) and kAStages dequantised A
+// stages (weight row m in lane m, two bf16 of K per column), which the MMAs
+// read in place: the weights never pass through shared memory, whose
+// bandwidth bounds the stage otherwise.
 template <bool GU>
 struct TcCfg {
     static constexpr int kRows = GU ? 2 * kM : kM;        // weight rows per item (gate rows, then up rows)
-    static constexpr int kBStages = 4;
+    static constexpr int kAStages = 4;                     // dequantised A stages in tensor memory
+    static constexpr int kACols = (GU ? 2 : 1) * (kKC / 2);   // TMEM columns of one A stage
+    static constexpr int kAccCols = (GU ? 2 : 1) * kN;        // accumulator columns
+    static constexpr uint32_t kTmemCols = GU ? 512 : 256;
+    static constexpr int kBStages = GU ? 6 : 4;
     static constexpr int kBTiles = GU ? 1 : 2;            // B tiles per stage: x, or h's hi and lo parts
     static constexpr int kBStageBytes = kBTiles * kTileBytes;
-    static constexpr int kABytes = (GU ? 2 : 1) * kTileBytes;
     static constexpr int kRawBytes = kRows * kRawW;
-    static constexpr int kBOff = 2 * kABytes;
+    static constexpr int kBOff = 0;
     static constexpr int kRawOff = kBOff + kBStages * kBStageBytes;
     static constexpr int kSmem = kRawOff + 2 * kRawBytes;
-    static constexpr int kDqWords = GU ? 4 : 2;             // nibble words a thread dequantises per stage
-    static_assert(kRows * 8 == kDqThr * kDqWords, "one dequantisation task per thread and stage");
-    static_assert(kBOff % 1024 == 0, "swizzled B tiles are 1024-byte aligned");
+    static constexpr int kDqK = GU ? 32 : 16;             // K elements a thread dequantises per stage
+    static_assert(kRows * kKC == kDqThr * kDqK, "one dequantisation task per thread and stage");
+    static_assert(kAccCols + kAStages * kACols <= (int)kTmemCols, "tensor memory columns");
+    static_assert(kAStages <= kBStages, "an A stage's release (the MMA commit of its stage) must still be "
+                                        "the barrier phase a dequantising warp can wait on");
 };
 static_assert(TcCfg<true>::kSmem <= 227 * 1024 - 2048 && TcCfg<false>::kSmem <= 227 * 1024 - 2048,
               "shared memory of the tensor-core kernels");
@@ -81,12 +87,6 @@ __device__ __forceinline__ void tl_stamp(const TcArgs &a, bool gu, int c, int s)
 {
     if (a.timeline && blockIdx.x == 0 && c < kTlStages)
         a.timeline[((gu ? 0 : 1) * kTlStages + c) * 8 + s] = globaltimer_ns();
-}
-
-// Offset of element (row, 8 * k8) of a no-swizzle 128 x kKC operand tile.
-__device__ __forceinline__ uint32_t tile_off(int row, int k8)
-{
-    return (uint32_t)(row >> 3) * kSbo + (uint32_t)(row & 7) * 16u + (uint32_t)k8 * kLbo;
 }
 
 // Two f32 in one 64-bit register (low word first) and back.
@@ -160,12 +160,15 @@ __device__ __forceinline__ int raw_window(int b) { return kBlockBytes * b - 8 * 
 //                re-targeted to the item's expert (tensormap.replace)
 //   B warp     - per stage, one 2-D TMA load of the 128 x 64 activation tile
 //                (pair-ordered, 128-byte swizzle) into a ring of B tiles
-//   16 warps   - per stage, dequantise their rows' nibble words from the raw
-//                buffer into one of two A buffers; the item's epilogue
-//   MMA warp   - per stage, the MMAs of the A buffer against the B tile
+//   16 warps   - per stage, dequantise a K slice of one weight row each (the
+//                row is the thread's TMEM lane) from the raw buffer into one of
+//                kAStages A stages in tensor memory (tcgen05.st); the item's
+//                epilogue
+//   MMA warp   - per stage, the MMAs of the A stage (tensor memory) against
+//                the B tile (shared memory)
 // Barriers (mbarriers): fullR/rfree per raw buffer, fullB/done per B tile,
-// aready per A buffer, tfree for the accumulators.  done[s] also frees the A
-// buffer of its stage.
+// aready per A stage, tfree for the accumulators.  done[s] also frees the A
+// stage of its stage.
 template <bool GU>
 __global__ void __launch_bounds__(kTcThr, 1)
     tc_kernel(const __grid_constant__ TcArgs a, const __grid_constant__ CUtensorMap bmap,
@@ -174,7 +177,8 @@ __global__ void __launch_bounds__(kTcThr, 1)
     using C = TcCfg<GU>;
     constexpr int RB = C::kBStages;
     extern __shared__ __align__(1024) uint8_t smem[];
-    __shared__ uint64_t fullB[RB], done_bar[RB], fullR[2], rfree[2], aready_bar[2], tfree_bar, fin_bar;
+    constexpr int NA = C::kAStages;
+    __shared__ uint64_t fullB[RB], done_bar[RB], fullR[2], rfree[2], aready_bar[NA], tfree_bar, fin_bar;
     __shared__ alignas(128) uint8_t s_map[128];
     __shared__ uint32_t tmem_slot;
     __shared__ int s_abort;
@@ -189,7 +193,7 @@ __global__ void __launch_bounds__(kTcThr, 1)
     volatile int *abortp = &s_abort;
 
     if (warp == 0) {
-        tmem_alloc(&tmem_slot, kTmemCols);
+        tmem_alloc(&tmem_slot, C::kTmemCols);
         tmem_relinquish();
     }
     if (tid == 0) {
@@ -200,8 +204,8 @@ __global__ void __launch_bounds__(kTcThr, 1)
         for (int q = 0; q < 2; ++q) {
             mbar_init(&fullR[q], 1);
             mbar_init(&rfree[q], kDqW);
-            mbar_init(&aready_bar[q], kDqW);
         }
+        for (int q = 0; q < NA; ++q) mbar_init(&aready_bar[q], kDqW);
         mbar_init(&tfree_bar, kDqW);
         mbar_init(&fin_bar, 1);
         // the swizzled B tiles need a 1024-byte aligned base
@@ -215,7 +219,6 @@ __global__ void __launch_bounds__(kTcThr, 1)
     __syncthreads();
     tc_fence_after_sync();
     const uint32_t tmem = tmem_slot;
-    uint8_t *const abuf = smem;
     uint8_t *const bbuf = smem + C::kBOff;
     uint8_t *const rbuf = smem + C::kRawOff;
 
@@ -312,27 +315,23 @@ __global__ void __launch_bounds__(kTcThr, 1)
         for (int c = 0; c < nchunks; ++c) {
             const int it = c / nK, kc = c - it * nK;
             if (kc == 0 && it > 0 && !tc_wait(a, &tfree_bar, (uint32_t)(it - 1) & 1u, abortp)) break;
-            if (!tc_wait(a, &aready_bar[c & 1], (uint32_t)(c >> 1) & 1u, abortp)) break;
+            if (!tc_wait(a, &aready_bar[c % NA], (uint32_t)(c / NA) & 1u, abortp)) break;
             if (!tc_wait(a, &fullB[c % RB], (uint32_t)(c / RB) & 1u, abortp)) break;
             tc_fence_after_sync();
             if (lane == 0) tl_stamp(a, GU, c, 5);
             if (lane == 0) {
-                // the A tile was written through the generic proxy by other
-                // threads and released to this one by aready; this proxy
-                // fence orders it before the MMAs' async-proxy reads
-                fence_proxy_async_smem();
-                const uint8_t *A = abuf + (c & 1) * C::kABytes;
+                // the A stage was written to tensor memory by other threads
+                // (tcgen05.st, waited for, fenced) and released by aready
+                const uint32_t A = tmem + (uint32_t)(C::kAccCols + (c % NA) * C::kACols);
                 const uint8_t *B = bbuf + (c % RB) * C::kBStageBytes;
 #pragma unroll
                 for (int ks = 0; ks < kKC / 16; ++ks) {
                     const uint64_t bd = umma_desc_sw128(B + 32 * ks);
-                    const uint64_t ad = umma_desc(A + 2 * ks * kLbo, kLbo, kSbo);
-                    umma_bf16(tmem, ad, bd, idesc, (kc | ks) != 0);
+                    umma_bf16_ts(tmem, A + 8 * ks, bd, idesc, (kc | ks) != 0);
                     if (GU)
-                        umma_bf16(tmem + kN, umma_desc(A + kTileBytes + 2 * ks * kLbo, kLbo, kSbo), bd,
-                                  idesc, (kc | ks) != 0);
+                        umma_bf16_ts(tmem + kN, A + kKC / 2 + 8 * ks, bd, idesc, (kc | ks) != 0);
                     else        // the same weights against h's lo part
-                        umma_bf16(tmem, ad, umma_desc_sw128(B + kTileBytes + 32 * ks), idesc, true);
+                        umma_bf16_ts(tmem, A + 8 * ks, umma_desc_sw128(B + kTileBytes + 32 * ks), idesc, true);
                 }
                 umma_commit(&done_bar[c % RB]);
                 tl_stamp(a, GU, c, 6);
@@ -342,12 +341,15 @@ __global__ void __launch_bounds__(kTcThr, 1)
         }
     } else {
         // ------------------------------------------------ dequantisation
-        // task: weight row drow, nibble words dw0 .. dw0 + kDqWords - 1 of the
-        // stage (each 8-lane phase stores one 128-byte core-matrix column)
-        const int drow = GU ? (lane & 7) + 8 * ((lane >> 3) + 4 * (warp >> 1))
-                            : (lane & 7) + 8 * ((lane >> 3) + 4 * (warp >> 2));
-        const int dw0 = GU ? 4 * (warp & 1) : 2 * (warp & 3);
-        uint8_t *const adst0 = abuf + (GU && drow >= kM ? kTileBytes : 0) + tile_off(drow & (kM - 1), 0);
+        // task: weight row 32 (warp % 4) + lane of the item (the thread's TMEM
+        // lane; gate/up: of the gate rows for warps 0..3 and 8..11, the up rows
+        // for 4..7 and 12..15), K elements kq * kDqK .. + kDqK - 1 of the stage
+        const int quarter = warp & 3;
+        const int mat = GU ? (warp >> 2) & 1 : 0;
+        const int kq = GU ? warp >> 3 : warp >> 2;
+        const int drow = mat * kM + 32 * quarter + lane;
+        const uint32_t a_lane = tmem + ((uint32_t)(32 * quarter) << 16) +
+                                (uint32_t)(C::kAccCols + mat * (kKC / 2) + kq * (C::kDqK / 2));
         int gs = -1;
 #pragma unroll 1
         for (int c = 0; c < nchunks; ++c) {
@@ -358,22 +360,37 @@ __global__ void __launch_bounds__(kTcThr, 1)
             if (j == 0) ++gs;                         // the stage opens a new raw buffer (HFQ4 block)
             if (j == 0 && !tc_wait(a, &fullR[gs & 1], (uint32_t)(gs >> 1) & 1u, abortp)) break;
             if (tl) tl_stamp(a, GU, c, 1);
-            // the MMAs of stage c - 2 are done: its A buffer is free
-            if (c >= 2 && !tc_wait(a, &done_bar[(c - 2) % RB], (uint32_t)((c - 2) / RB) & 1u, abortp)) break;
+            // the MMAs of stage c - NA are done: its A stage is free
+            if (c >= NA && !tc_wait(a, &done_bar[(c - NA) % RB], (uint32_t)((c - NA) / RB) & 1u, abortp)) break;
+            tc_fence_after_sync();
             if (tl) tl_stamp(a, GU, c, 2);
             const uint8_t *raw = rbuf + (gs & 1) * C::kRawBytes + drow * kRawW + 8 * (b & 1);
             const float2 sz = *reinterpret_cast<const float2 *>(raw);
-            const uint8_t *pw = raw + 8 + 32 * j + 4 * dw0;
-            uint8_t *ad = adst0 + (c & 1) * C::kABytes;
+            const uint8_t *pw = raw + 8 + 32 * j + kq * (C::kDqK / 2);
+            const uint32_t at = a_lane + (uint32_t)((c % NA) * C::kACols);
+            if (GU) {
+                uint32_t v[16];
 #pragma unroll
-            for (int h = 0; h < C::kDqWords / 2; ++h) {
-                const uint2 w = *reinterpret_cast<const uint2 *>(pw + 8 * h);
-                *reinterpret_cast<uint4 *>(ad + (dw0 + 2 * h) * kLbo) = deq8(w.x, sz.x, sz.y);
-                *reinterpret_cast<uint4 *>(ad + (dw0 + 2 * h + 1) * kLbo) = deq8(w.y, sz.x, sz.y);
+                for (int h = 0; h < 2; ++h) {
+                    const uint2 w = *reinterpret_cast<const uint2 *>(pw + 8 * h);
+                    const uint4 d0 = deq8(w.x, sz.x, sz.y), d1 = deq8(w.y, sz.x, sz.y);
+                    v[8 * h + 0] = d0.x; v[8 * h + 1] = d0.y; v[8 * h + 2] = d0.z; v[8 * h + 3] = d0.w;
+                    v[8 * h + 4] = d1.x; v[8 * h + 5] = d1.y; v[8 * h + 6] = d1.z; v[8 * h + 7] = d1.w;
+                }
+                tmem_st16(at, v);
+            } else {
+                uint32_t v[8];
+                const uint2 w = *reinterpret_cast<const uint2 *>(pw);
+                const uint4 d0 = deq8(w.x, sz.x, sz.y), d1 = deq8(w.y, sz.x, sz.y);
+                v[0] = d0.x; v[1] = d0.y; v[2] = d0.z; v[3] = d0.w;
+                v[4] = d1.x; v[5] = d1.y; v[6] = d1.z; v[7] = d1.w;
+                tmem_st8(at, v);
             }
+            tmem_st_wait();
+            tc_fence_before_sync();
             __syncwarp();
             if (lane == 0) {
-                mbar_arrive(&aready_bar[c & 1]);
+                mbar_arrive(&aready_bar[c % NA]);
                 if (j == 3 || kc == nK - 1) mbar_arrive(&rfree[gs & 1]);   // raw buffer read
             }
             if (tl) tl_stamp(a, GU, c, 3);
@@ -423,7 +440,7 @@ __global__ void __launch_bounds__(kTcThr, 1)
     tc_fence_before_sync();
     __syncthreads();
     tc_fence_after_sync();
-    if (warp == 0) tmem_dealloc(tmem, kTmemCols);
+    if (warp == 0) tmem_dealloc(tmem, C::kTmemCols);
 }
 
 // Work items per expert: ceil(cnt/kN) token tiles x (rows/kM) row tiles, for
