@@ -144,11 +144,11 @@ class ClockSampler:
 
 # ------------------------------------------------------------ link probes
 
-def measure_pcie(torch, eo, nbytes=1 << 30):
+def measure_pcie(torch, eo, nbytes=1 << 30, flags=0):
     """Host-to-device bandwidth two ways: a pinned cudaMemcpy and the zero-copy
     read kernel over a mapped arena (the strata report's link probe, done here
     with the expert kernel's own load path)."""
-    h, d = eo.hfq_host_arena_create(nbytes)
+    h, d = eo.hfq_host_arena_create(nbytes, flags)
     try:
         sink = torch.zeros(1, dtype=torch.int64, device="cuda")
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -245,11 +245,13 @@ class StackInputs:
     """G token groups of a stack workload: logits [G, L, T, E] and inputs
     [G, T, H] (bf16), on the device, plus each group's streamed bytes."""
 
-    def __init__(self, torch, W, w, L, T, G):
+    def __init__(self, torch, W, w, L, T, G, token0=0):
         import numpy as np
-        self.logits = np.stack([np.stack([W.logits(w, l, g * T, T) for l in range(L)])
-                                for g in range(G)])
-        self.xs = np.stack([W.activations(w, g * T, T)[0] for g in range(G)])
+        # one generator call per layer for all G * T tokens (token g * T + t of
+        # group g), the same values as per-group calls
+        lg = np.stack([W.logits(w, l, token0, G * T) for l in range(L)])       # [L, G*T, E]
+        self.logits = np.ascontiguousarray(lg.reshape(L, G, T, -1).transpose(1, 0, 2, 3))
+        self.xs = W.activations(w, token0, G * T)[0].reshape(G, T, -1)
         self.d_logits = torch.from_numpy(self.logits).cuda()
         self.d_x = torch.from_numpy(self.xs.view(np.int16)).cuda()
         self.G, self.T = G, T
@@ -539,6 +541,23 @@ def run_verify_suite(args, K, W_):
     return res
 
 
+def thp_state():
+    """The kernel's transparent-huge-page mode and the anonymous huge pages in
+    use now (kB), as the system reports them."""
+    out = {}
+    try:
+        out["mode"] = open("/sys/kernel/mm/transparent_hugepage/enabled").read().strip()
+    except OSError:
+        out["mode"] = "unknown"
+    try:
+        for line in open("/proc/meminfo"):
+            if line.startswith("AnonHugePages:"):
+                out["anon_huge_kb"] = int(line.split()[1])
+    except OSError:
+        pass
+    return out
+
+
 class DualModel:
     """Every expert of a model twice: packed in HBM and in one pinned, mapped
     host arena, at the same offset (layer * E + expert) * expert_bytes.  A
@@ -617,10 +636,162 @@ def run_offload_suite(args, K, W_):
                  "hbm_expert_bytes": hn, "host_expert_bytes": hs,
                  "host_pages": "2 MiB (madvise)" if args.hugepage else "4 KiB"})
             timer.close()
+    res.update(run_cache_suite(args, torch, eo, dual, w, K, W_, bw_pcie, peak, peak_kind))
     dual.close()
+    # host arena page size (Strata report, pitfall 7): the all-host row again,
+    # with the arena on 2 MiB transparent huge pages (madvise, then registered)
+    if not args.hugepage:
+        before = thp_state()
+        dual = DualModel(torch, eo, store, hugepage=True)
+        after = thp_state()
+        pcie2 = measure_pcie(torch, eo, flags=eo.ARENA_HUGEPAGE)
+        loc, _, hn, hs = eo.hfq_placement_build(counts, eb, 0, 0, 170 * 2**30)
+        layers = dual.layers(loc)
+        per_group = [step_bytes(inp.logits[g], k, eb, loc) for g in range(inp.G)]
+        timer = StackTimer(torch, eo, layers, inp, k, H, I, E)
+        steps = max(5, K // 4)
+        total_ms, per_launch, clocks = timer.run(steps, max(3, W_ // 4))
+        hbm_b = sum(per_group[i % inp.G][0] for i in range(steps)) / steps
+        host_b = sum(per_group[i % inp.G][1] for i in range(steps)) / steps
+        roof = offload_roofline(inp.logits, k, eb, loc, hbm_b, host_b, sum(per_launch) / steps,
+                                peak, peak_kind, max(pcie2.values()), pcie2, kernel_name(1, 1))
+        roof.pop("pcie")
+        res["offload_n0_h0_hugepage"] = sub_result(
+            1, steps, total_ms, per_launch, clocks, roof, 1,
+            {"workload": w.name, "resident_layers": 0, "hot_per_layer": 0,
+             "host_pages": "2 MiB transparent huge pages asked for (madvise)",
+             "pcie_hugepage_arena": pcie2, "thp_before": before, "thp_after_arena": after})
+        timer.close()
+        dual.close()
     store.close()
     del store, dual
     torch.cuda.empty_cache()
+    return res
+
+
+def run_cache_suite(args, torch, eo, dual, w, K, W_, bw_pcie, peak, peak_kind):
+    """Every expert of the 48 x 512 model in pinned host memory (N = 0), with
+    a dynamic VRAM expert cache in front of it (Strata report, "model and
+    engine") and, for comparison, with copy-engine staging of each layer's
+    selected experts before the layer runs (the alternative the hipfire
+    offload explainer's "PCIe pass-through" section argues against).
+
+    Cache: after each step the step's routing (idx_all, copied to the host)
+    goes to hfq_cache_observe layer by layer, which admits up to 4 missed
+    experts per layer (frequency policy) with the copy engine; misses are read
+    zero-copy meanwhile.  A step is the stack kernel plus that host round
+    trip; every step routes a new token (skewed routing, 51 hot experts of
+    512 per layer).  Staging: per layer, route on the device, copy the ids to
+    the host, copy the selected experts into 8 HBM slots, run the layer."""
+    import time
+
+    import numpy as np
+
+    from synth import workloads as W
+    L, E, H, I, k = w.layers, w.experts, w.hidden, w.inter, w.top_k
+    eb = dual.store.eb
+    offs = (np.arange(L * E, dtype=np.uint64) * np.uint64(eb)).reshape(L, E)
+    home = offs + np.uint64(dual.host_dev)
+    host_src = offs + np.uint64(dual.host)
+    home_loc = np.ones((L, E), np.uint8)
+    warm, timed = max(64, 8 * W_), max(32, K)
+    inp = StackInputs(torch, W, w, L, 1, warm + timed, token0=1 << 20)
+    stream = torch.cuda.current_stream()
+    ws = torch.zeros(eo.hfq4_stack_workspace_bytes(1, k, H, I, E), dtype=torch.uint8, device="cuda")
+    x_out = torch.empty((1, H), dtype=torch.int16, device="cuda")
+    idx_all = torch.empty((L, 1, k), dtype=torch.int32, device="cuda")
+    wts_all = torch.empty((L, 1, k), dtype=torch.float32, device="cuda")
+    idx_host = torch.empty((L, 1, k), dtype=torch.int32).pin_memory()
+    res = {}
+    for slots in (51, 128):
+        slot_mem = torch.empty(L * slots * eb, dtype=torch.uint8, device="cuda")
+        table = torch.empty(L * E, dtype=torch.int64, device="cuda")
+        locd = torch.empty(L * E, dtype=torch.uint8, device="cuda")
+        cache = eo.ExpertCache(L, E, eb, slots, home, host_src, home_loc, slot_mem, table, locd, stream)
+        layers = [eo.Layer(table[l * E:(l + 1) * E], E, H, I, expert_loc=locd[l * E:(l + 1) * E])
+                  for l in range(L)]
+        arr = eo.layer_array(layers)
+        kern_ms = []
+
+        def step(g, timed_step):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            eo.hfq4_moe_decode_stack(layers, inp.d_logits[g], k, inp.d_x[g], 1, x_out, ws,
+                                     idx_all=idx_all, wts_all=wts_all, _layer_array=arr)
+            e1.record()
+            idx_host.copy_(idx_all, non_blocking=True)
+            torch.cuda.synchronize()
+            if timed_step:
+                kern_ms.append(e0.elapsed_time(e1))
+            ids = idx_host.numpy()
+            for l in range(L):
+                cache.observe(l, ids[l].ravel(), 4)
+
+        for g in range(warm):
+            step(g, False)
+        before = cache.stats()
+        sampler = ClockSampler(0)
+        sampler.start()
+        t0 = time.perf_counter()
+        for g in range(warm, warm + timed):
+            step(g, True)
+        torch.cuda.synchronize()
+        dt = time.perf_counter() - t0
+        clocks = sampler.stop()
+        after = cache.stats()
+        eo.hfq_workspace_status(ws)
+        hits, misses = after["hits"] - before["hits"], after["misses"] - before["misses"]
+        res[f"offload_n0_cache{slots}"] = {
+            "value": round(timed / dt, 2), "unit": "tokens/s", "ms_per_step": round(dt / timed * 1e3, 4),
+            "steps": timed, "tokens_per_step": 1, "workload": w.name,
+            "timing": "host wall clock per step: stack kernel + idx copy + cache update (copy engine)",
+            "cache_slots_per_layer": slots, "hit_rate": round(hits / max(1, hits + misses), 4),
+            "admitted_per_step": round((after["admitted"] - before["admitted"]) / timed, 3),
+            "kernel_ms_per_step": round(sum(kern_ms) / len(kern_ms), 4),
+            "warmup_steps": warm, "gpu_launches": timed, "clocks": clocks}
+        cache.close()
+        del slot_mem, table, locd
+    # staging before use: per layer route, copy ids to the host, stage, run
+    slots = k
+    slot_mem = torch.empty(L * slots * eb, dtype=torch.uint8, device="cuda")
+    table = torch.empty(L * E, dtype=torch.int64, device="cuda")
+    locd = torch.empty(L * E, dtype=torch.uint8, device="cuda")
+    cache = eo.ExpertCache(L, E, eb, slots, home, host_src, home_loc, slot_mem, table, locd, stream)
+    layers = [eo.Layer(table[l * E:(l + 1) * E], E, H, I, expert_loc=locd[l * E:(l + 1) * E])
+              for l in range(L)]
+    idx1 = torch.empty((1, k), dtype=torch.int32, device="cuda")
+    w1 = torch.empty((1, k), dtype=torch.float32, device="cuda")
+    idx1_host = torch.empty((1, k), dtype=torch.int32).pin_memory()
+    xa = torch.empty((1, H), dtype=torch.int16, device="cuda")
+    xb = torch.empty((1, H), dtype=torch.int16, device="cuda")
+
+    def staged_token(g):
+        cur = inp.d_x[g]
+        for l in range(L):
+            eo.moe_route(inp.d_logits[g, l], 1, E, k, idx1, w1)
+            idx1_host.copy_(idx1, non_blocking=True)
+            torch.cuda.synchronize()
+            cache.observe(l, idx1_host.numpy().ravel(), -1)
+            nxt = xa if l % 2 == 0 else xb
+            eo.hfq4_moe_decode_stack(layers[l:l + 1], inp.d_logits[g, l], k, cur, 1, nxt, ws)
+            cur = nxt
+        torch.cuda.synchronize()
+
+    n_staged = max(3, min(8, K // 4))
+    for g in range(2):
+        staged_token(g)
+    t0 = time.perf_counter()
+    for g in range(2, 2 + n_staged):
+        staged_token(g)
+    dt = time.perf_counter() - t0
+    eo.hfq_workspace_status(ws)
+    res["offload_n0_staged"] = {
+        "value": round(n_staged / dt, 2), "unit": "tokens/s", "ms_per_step": round(dt / n_staged * 1e3, 4),
+        "steps": n_staged, "tokens_per_step": 1, "workload": w.name,
+        "timing": "host wall clock per token: per layer route + idx copy + copy-engine staging of the "
+                  "selected experts + the layer",
+        "pcie_gbs_measured": bw_pcie, "gpu_launches": 2 * L * n_staged}
+    cache.close()
     return res
 
 

@@ -63,6 +63,9 @@ _SIGS = {
     "hfq4_stack_launches": (_i, [_i, _i, _i, _i, _i]),
     "hfq4_moe_decode_stack": (_i, [ctypes.POINTER(hfq4_layer), _i, _vp, _i, _vp, _i, _vp, _vp,
                                    _vp, _vp, _i, _vp, _sz, _vp]),
+    "moe_router_logits": (_i, [_vp, _i, _i, _i, _vp, _i, _i, _vp, _vp]),
+    "hfq4_moe_decode_stack_routed": (_i, [ctypes.POINTER(hfq4_layer), _i, _vp, _i, _i, _vp, _i,
+                                          _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
     "hfq_workspace_status": (_i, [_vp, _sz, _vp]),
     "hfq_set_option": (_i, [_i, ctypes.c_longlong]),
     "hfq_host_arena_create": (_i, [_sz, _i, ctypes.POINTER(_vp), ctypes.POINTER(_vp)]),
@@ -71,6 +74,13 @@ _SIGS = {
                                  ctypes.POINTER(_sz), ctypes.POINTER(_sz)]),
     "hfq_placement_pointers": (_i, [_i, _i, _sz, _vp, _vp, _vp, _vp, _vp]),
     "hfq_probe_read": (_i, [_vp, _sz, _i, _vp, _vp]),
+    "hfq_cache_create": (_i, [_i, _i, _sz, _i, _vp, _vp, _vp, _vp, _sz, _vp, _vp, _vp,
+                              ctypes.POINTER(_vp)]),
+    "hfq_cache_observe": (_i, [_vp, _i, _vp, _i, _i, _vp]),
+    "hfq_cache_slot_of": (_i, [_vp, _i, _i, ctypes.POINTER(_i)]),
+    "hfq_cache_stats": (_i, [_vp, ctypes.POINTER(_u64), ctypes.POINTER(_u64), ctypes.POINTER(_u64),
+                             ctypes.POINTER(_u64)]),
+    "hfq_cache_destroy": (_i, [_vp]),
 }
 
 _lib = None
@@ -175,6 +185,13 @@ def moe_route(logits, T: int, E: int, k: int, idx, wts, cnt=None, off=None, perm
                            _ptr(perm), _ptr(workspace), ws_bytes, _stream(stream)))
 
 
+def moe_router_logits(x, x_dtype: int, T: int, hidden: int, router, router_dtype: int,
+                      n_experts: int, logits, stream=None) -> None:
+    """logits [T, E] f32 = x Wr^T on the device."""
+    _check(lib().moe_router_logits(_ptr(x), x_dtype, T, hidden, _ptr(router), router_dtype,
+                                   n_experts, _ptr(logits), _stream(stream)))
+
+
 # ---------------------------------------------------------------- forward
 
 class Layer:
@@ -229,6 +246,17 @@ def hfq4_moe_decode_stack(layers, logits, k: int, x0, T: int, x_out, workspace, 
     _check(lib().hfq4_moe_decode_stack(arr, len(layers), _ptr(logits), k, _ptr(x0), T, _ptr(x_out),
                                        _ptr(y_all), _ptr(idx_all), _ptr(wts_all), path,
                                        _ptr(workspace), _nbytes(workspace), _stream(stream)))
+
+
+def hfq4_moe_decode_stack_routed(layers, router, router_dtype: int, k: int, x0, T: int, x_out,
+                                 workspace, y_all=None, idx_all=None, wts_all=None,
+                                 logits_all=None, stream=None, _layer_array=None) -> None:
+    arr = _layer_array if _layer_array is not None else layer_array(layers)
+    _check(lib().hfq4_moe_decode_stack_routed(arr, len(layers), _ptr(router), router_dtype, k,
+                                              _ptr(x0), T, _ptr(x_out), _ptr(y_all),
+                                              _ptr(idx_all), _ptr(wts_all), _ptr(logits_all),
+                                              _ptr(workspace), _nbytes(workspace),
+                                              _stream(stream)))
 
 
 OPT_WAIT_TIMEOUT_NS, OPT_TEST_MISSING_ARRIVALS, OPT_TIMELINE_BUFFER = 1, 2, 3
@@ -289,3 +317,52 @@ def hfq_placement_pointers(loc, slot, expert_bytes: int, hbm_base: int, host_dev
 
 def hfq_probe_read(src, nbytes: int, iters: int, sink, stream=None) -> None:
     _check(lib().hfq_probe_read(_ptr(src), nbytes, iters, _ptr(sink), _stream(stream)))
+
+
+# ------------------------------------------------------------ expert cache
+
+class ExpertCache:
+    """hfq_cache_* over the pointer (and location) tables of L layers.
+
+    home, host_src: uint64 [L, E] numpy arrays (see include/hfq4moe.h);
+    home_loc: uint8 [L, E]; slot_mem, table_dev, loc_dev: device tensors or
+    None (table_dev None: bookkeeping only)."""
+
+    def __init__(self, L: int, E: int, expert_bytes: int, slots: int, home, host_src, home_loc,
+                 slot_mem=None, table_dev=None, loc_dev=None, stream=None):
+        import numpy as np
+        self._keep = [np.ascontiguousarray(home, np.uint64), np.ascontiguousarray(host_src, np.uint64),
+                      np.ascontiguousarray(home_loc, np.uint8)]
+        h = ctypes.c_void_p()
+        _check(lib().hfq_cache_create(L, E, expert_bytes, slots, self._keep[0].ctypes.data,
+                                      self._keep[1].ctypes.data, self._keep[2].ctypes.data,
+                                      _ptr(slot_mem), _nbytes(slot_mem) if slot_mem is not None else 0,
+                                      _ptr(table_dev), _ptr(loc_dev), _stream(stream), ctypes.byref(h)))
+        self.handle = h.value
+
+    def observe(self, layer: int, ids, max_admit: int, stream=None) -> None:
+        import numpy as np
+        a = np.ascontiguousarray(ids, np.int32).ravel()
+        _check(lib().hfq_cache_observe(self.handle, layer, a.ctypes.data, a.size, max_admit,
+                                       _stream(stream)))
+
+    def slot_of(self, layer: int, expert: int) -> int:
+        s = ctypes.c_int()
+        _check(lib().hfq_cache_slot_of(self.handle, layer, expert, ctypes.byref(s)))
+        return s.value
+
+    def stats(self):
+        v = [ctypes.c_uint64() for _ in range(4)]
+        _check(lib().hfq_cache_stats(self.handle, *[ctypes.byref(x) for x in v]))
+        return dict(zip(("hits", "misses", "admitted", "evicted"), (x.value for x in v)))
+
+    def close(self) -> None:
+        if self.handle:
+            _check(lib().hfq_cache_destroy(self.handle))
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except (HfqError, AttributeError, TypeError):
+            pass

@@ -9,9 +9,10 @@
 //   1. the eight warps route the token (each the top k of an eighth of the
 //      experts, warp 0 merging; softmax top-k, renormalised; hipfire offload
 //      explainer, opening section), reading layer l's logits only after layer
-//      l-1 has finished everywhere, and warp 0 at once issues the 3k bulk copies
-//      (1-D TMA, no multicast), lane j for slot j, into k fixed shared-memory
-//      slots with one mbarrier for gate/up and one for down per slot.  Experts
+//      l-1 has finished everywhere, and warp 0 at once issues the 2k gate/up
+//      bulk copies (1-D TMA, no multicast), lane j for slot j, into k fixed
+//      shared-memory slots with one mbarrier for gate/up and one for down per
+//      slot; warp j issues slot j's down copy once its gate/up bytes are in.  Experts
 //      in host memory are read by the owning warp with 16-byte loads over PCIe
 //      (hipfire offload explainer, "PCIe pass-through").  Warps 1..7 prepare
 //      their activation registers meanwhile.
@@ -56,7 +57,10 @@ constexpr int kSmemOptin = 232448;      // 227 KB per CTA on sm_100
 struct D1Args {
     const void *const *eptr[HFQ_MAX_STACK_LAYERS];
     const uint8_t *eloc[HFQ_MAX_STACK_LAYERS];
-    const float *logits;      // [L][E], or null when the routing is given
+    const float *logits;      // [L][E], or null when the routing is given or computed
+    const uint16_t *router;   // [L][E][H] bf16 router weights: logits = Wr x_l in the kernel, or null
+    uint64_t *lbuf;           // [2][E] {f32 logit, tag} words (router): each CTA computes E/G logits
+    float *logits_out;        // [L][E] the computed logits (router), or null
     const int32_t *idx_in;    // [k] given routing (single layer), or null
     const float *wts_in;
     const void *x0;           // [H] bf16 (f32 when x0_f32)
@@ -76,7 +80,7 @@ struct D1Args {
                               // expect a tag nobody writes
     // shared-memory layout, bytes; a slot is [gate span][up span][down span]
     int slot_bytes, up_off, down_off;
-    int xs_off, ptab_off, ltab_off, ysh_off, sh_off;
+    int xs_off, ptab_off, ltab_off, ysh_off, lsm_off, sh_off;
     int ltab_stride;
 };
 
@@ -109,11 +113,12 @@ __device__ __forceinline__ uint32_t xch_tag(uint32_t epoch, int l)
 }
 
 // Signature of the exchange layout: bit 31 set (0 means none), k, padded I,
-// H and whether x is exchanged (several layers).
-__host__ __device__ __forceinline__ uint32_t xch_signature(int k, int Ip, int H, int L)
+// H, whether x is exchanged (several layers) and the logit exchange's E (0
+// without the in-kernel router).
+__host__ __device__ __forceinline__ uint32_t xch_signature(int k, int Ip, int H, int L, int E_router)
 {
-    return 0x80000000u | ((uint32_t)k << 24) | ((uint32_t)(Ip >> 8) << 20) | ((uint32_t)(H >> 3) << 8) |
-           (L > 1 ? 1u : 0u);
+    return 0x80000000u | ((uint32_t)k << 26) | ((uint32_t)(Ip >> 8) << 23) | ((uint32_t)(H >> 7) << 18) |
+           ((uint32_t)E_router << 1) | (L > 1 ? 1u : 0u);
 }
 
 
@@ -226,10 +231,11 @@ __global__ void __launch_bounds__(kThr, 1) decode1_kernel(const __grid_constant_
     uint8_t *ptab = smem + a.ptab_off;                                // [2][E] addresses
     uint8_t *ltab = smem + a.ltab_off;                                // [2][ltab_stride]
     float *ysh = reinterpret_cast<float *>(smem + a.ysh_off);        // [kW][kMaxDRows]
+    float *lsm = reinterpret_cast<float *>(smem + a.lsm_off);        // [E] logits (router)
     D1Shared &sh = *reinterpret_cast<D1Shared *>(smem + a.sh_off);
     const WaitCtx wc{a.ctl, a.timeout_ns, &sh.abort};
     const uint32_t epoch = *(volatile const unsigned *)(a.ctl + kCtlEpoch);
-    const uint32_t sig = xch_signature(k, Ip, H, a.L);
+    const uint32_t sig = xch_signature(k, Ip, H, a.L, a.router ? E : 0);
     const bool reset = *(volatile const unsigned *)(a.ctl + kCtlSig) != sig;
 
     if (tid == 0) {
@@ -247,9 +253,11 @@ __global__ void __launch_bounds__(kThr, 1) decode1_kernel(const __grid_constant_
         // another exchange layout ran last on these buffers: zero them (tag 0
         // matches no launch) and wait until every CTA has done its share
         const size_t nh = (size_t)2 * k * Ip, nx = a.L > 1 && a.xbuf ? (size_t)2 * H : 0;
-        for (size_t i = (size_t)c * kThr + tid; i < nh + nx; i += (size_t)G * kThr) {
+        const size_t nl = a.router ? (size_t)2 * E : 0;
+        for (size_t i = (size_t)c * kThr + tid; i < nh + nx + nl; i += (size_t)G * kThr) {
             if (i < nh) a.h[i] = 0ull;
-            else a.xbuf[i - nh] = 0ull;
+            else if (i < nh + nx) a.xbuf[i - nh] = 0ull;
+            else a.lbuf[i - nh - nx] = 0ull;
         }
         __syncthreads();
         if (tid == 0) {
@@ -321,10 +329,67 @@ __global__ void __launch_bounds__(kThr, 1) decode1_kernel(const __grid_constant_
         }
         if (__syncthreads_or(sh.abort)) break;
         stamp(a, l, 4);
+        // ---------------------------------------------- 1a'. router (optional)
+        // logits = Wr_l x_l: CTA c computes experts [c E / G, (c + 1) E / G),
+        // one warp each (the order of moe_router_logits, same bits), writes
+        // them as tagged words, and every CTA polls all E of them into lsm
+        if (a.router && !a.idx_in) {
+            const int r_lo = (int)((long long)c * E / G), r_hi = (int)((long long)(c + 1) * E / G);
+            const uint32_t tag = xch_tag(epoch, l);
+            for (int e = r_lo + warp; e < r_hi; e += kW) {
+                const uint16_t *row = a.router + ((size_t)l * E + e) * H;
+                float acc = 0.0f;
+                for (int h0 = 8 * lane; h0 < H; h0 += 256) {
+                    const uint4 v = ld_nc_v4(row + h0);
+                    const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        acc = fmaf(xs[xp4(h0 + 2 * i)], __uint_as_float(w4[i] << 16), acc);
+                        acc = fmaf(xs[xp4(h0 + 2 * i + 1)], __uint_as_float(w4[i] & 0xFFFF0000u), acc);
+                    }
+                }
+                acc = warp_sum(acc);
+                if (lane == 0) st_tagged(a.lbuf + (size_t)(l & 1) * E + e, acc, tag);
+            }
+            // poll: thread tid reads logits tid and tid + kThr (E <= 512)
+            const uint64_t *lw = a.lbuf + (size_t)(l & 1) * E;
+            unsigned pend = (tid < E ? 1u : 0u) | (tid + kThr < E ? 2u : 0u);
+            uint64_t t0 = 0;
+            for (int it = 0; pend; ++it) {
+                uint64_t v[2] = {0ull, 0ull};
+#pragma unroll
+                for (int m = 0; m < 2; ++m)
+                    if (pend >> m & 1u)
+                        asm volatile("ld.relaxed.gpu.global.b64 %0, [%1];" : "=l"(v[m]) : "l"(lw + tid + kThr * m) : "memory");
+#pragma unroll
+                for (int m = 0; m < 2; ++m)
+                    if ((pend >> m & 1u) && (uint32_t)(v[m] >> 32) == tag) {
+                        lsm[tid + kThr * m] = __uint_as_float((uint32_t)v[m]);
+                        pend &= ~(1u << m);
+                    }
+                if (it == 16) t0 = globaltimer_ns();
+                if (pend && it > 16 && (it & 15) == 0) {
+                    if (sh.abort || *(volatile unsigned *)a.ctl != 0u) {
+                        sh.abort = 1;
+                        break;
+                    }
+                    if (deadline_passed(t0, a.timeout_ns)) {
+                        raise_timeout(wc);
+                        break;
+                    }
+                }
+            }
+            if (__syncthreads_or(sh.abort)) break;
+            if (a.logits_out && c == 0)
+                for (int e = tid; e < E; e += kThr) a.logits_out[(size_t)l * E + e] = lsm[e];
+        }
         // ---------------------------------------------- 1b. route (all warps)
         int re = -1;
         float rw = 0.0f;
-        if (!a.idx_in) cta_route<kW>(a.logits + (size_t)l * E, E, k, sh.cand_key, sh.cand_e, re, rw);
+        if (!a.idx_in) {
+            if (a.router) cta_route<kW, true>(lsm, E, k, sh.cand_key, sh.cand_e, re, rw);
+            else cta_route<kW>(a.logits + (size_t)l * E, E, k, sh.cand_key, sh.cand_e, re, rw);
+        }
         if (warp == 0) {
             // ------------------------------------------ 1c. issue copies
             cp_async_wait_all();
@@ -378,7 +443,6 @@ __global__ void __launch_bounds__(kThr, 1) decode1_kernel(const __grid_constant_
                     uint8_t *slot = slots + (size_t)lane * a.slot_bytes;
                     if (sg.len) bulk_g2s_hint(slot, base + sg.src, (uint32_t)sg.len, &sh.gu_bar[lane], pol);
                     if (su.len) bulk_g2s_hint(slot + a.up_off, base + su.src, (uint32_t)su.len, &sh.gu_bar[lane], pol);
-                    if (sd.len) bulk_g2s_hint(slot + a.down_off, base + sd.src, (uint32_t)sd.len, &sh.d_bar[lane], pol);
                 }
                 if (lane == 0) { sh.armed = l + 1; sh.hostmask = hm; }
                 __syncwarp();
@@ -430,6 +494,12 @@ __global__ void __launch_bounds__(kThr, 1) decode1_kernel(const __grid_constant_
             } else if (!wait_mbar_phase(wc, &sh.gu_bar[j], par)) {
                 ok = false;
                 break;
+            } else if (lane == 0 && sd.len) {
+                // the slot's down rows, now that its gate/up bytes are in; the
+                // span was last read by the generic proxy (previous layer)
+                fence_proxy_async_smem();
+                bulk_g2s_hint(slot + a.down_off, sh.base[j] + sd.src, (uint32_t)sd.len, &sh.d_bar[j],
+                              l2_evict_first_policy());
             }
             stamp_dep(a, l, 5 + j, lane == 0 && (warp == 0 || warp == 7), 0.f);
             const uint8_t *g0 = slot + sg.delta, *u0 = slot + a.up_off + su.delta;
@@ -676,7 +746,7 @@ hfq_status decode1_launch(const hfq4_layer *layers, int L, const float *logits, 
                           const float *wts_in, const void *x0, bool x0_f32, int k, uint16_t *x_out,
                           uint16_t *xbuf, float *h, float *y, uint16_t *y_bf16, int32_t *idx_all,
                           float *wts_all, unsigned *ctl, long long timeout_ns, int extra_arrivals,
-                          cudaStream_t s)
+                          cudaStream_t s, const uint16_t *router, uint64_t *lbuf, float *logits_out)
 {
     const int H = layers[0].hidden, I = layers[0].inter, E = layers[0].n_experts;
     const int G = sm_count();
@@ -699,7 +769,9 @@ hfq_status decode1_launch(const hfq4_layer *layers, int L, const float *logits, 
         a.eptr[l] = layers[l].expert_ptr;
         a.eloc[l] = layers[l].expert_loc;
     }
+    if (router && (!lbuf || !aligned16(router) || H % 8)) return HFQ_ERR_UNSUPPORTED;
     a.logits = logits; a.idx_in = idx_in; a.wts_in = wts_in; a.x0 = x0; a.x_out = x_out;
+    a.router = router; a.lbuf = lbuf; a.logits_out = logits_out;
     a.xbuf = reinterpret_cast<uint64_t *>(xbuf); a.h = reinterpret_cast<uint64_t *>(h); a.y = y; a.y_bf16 = y_bf16; a.idx_all = idx_all; a.wts_all = wts_all;
     a.ctl = ctl; a.timeout_ns = timeout_ns; a.extra_arrivals = extra_arrivals;
     a.timeline = static_cast<unsigned long long *>(option_timeline());
@@ -726,6 +798,8 @@ hfq_status decode1_launch(const hfq4_layer *layers, int L, const float *logits, 
     off += (size_t)2 * a.ltab_stride;
     a.ysh_off = (int)off;
     off += (size_t)kW * kMaxDRows * 4;
+    a.lsm_off = (int)off;
+    off += router ? up16((size_t)E * 4) : 0;
     a.sh_off = (int)up16(off);
     const size_t smem = (size_t)a.sh_off + sizeof(D1Shared);
 

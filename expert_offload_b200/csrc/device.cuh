@@ -107,11 +107,15 @@ hfq_status launch_stack(const hfq4_layer *layers, int L, const float *logits, co
 // Persistent decode kernel for one token (decode1.cu); launch_stack hands T = 1
 // to it when decode1_launch accepts the shape (else HFQ_ERR_UNSUPPORTED with no
 // launch, and the general kernel runs).
+// With `router` (bf16 [L][E][H]) the kernel computes each layer's logits
+// from x_l itself (`lbuf`: [2][E] exchange words in the workspace;
+// `logits_out`: optional [L][E] copy of them) instead of reading `logits`.
 hfq_status decode1_launch(const hfq4_layer *layers, int L, const float *logits, const int32_t *idx_in,
                           const float *wts_in, const void *x0, bool x0_f32, int k, uint16_t *x_out,
                           uint16_t *xbuf, float *h, float *y, uint16_t *y_bf16, int32_t *idx_all,
                           float *wts_all, unsigned *ctl, long long timeout_ns, int extra_arrivals,
-                          cudaStream_t s);
+                          cudaStream_t s, const uint16_t *router = nullptr, uint64_t *lbuf = nullptr,
+                          float *logits_out = nullptr);
 // Persistent decode kernel for 2..8 tokens (verify.cu); launch_stack hands such
 // batches to it when verify_launch accepts the shape (else HFQ_ERR_UNSUPPORTED
 // with no launch, and the general kernel runs).
@@ -121,6 +125,10 @@ hfq_status verify_launch(const hfq4_layer *layers, int L, const float *logits, c
                          float *wts_all, unsigned *ctl, long long timeout_ns, int extra_arrivals,
                          cudaStream_t s);
 int sm_count();
+
+// Router GEMV logits = x Wr^T for T tokens (pack_route.cu).
+hfq_status launch_router(const void *x, bool x_bf16, const void *wr, bool wr_bf16, int T, int E, int H,
+                         float *logits, cudaStream_t s);
 
 // Tensor-core expert path (tc.cu).
 size_t tc_workspace_bytes(int T, int k, int H, int I, int E);

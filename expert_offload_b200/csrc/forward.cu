@@ -336,8 +336,10 @@ hfq_status hfq4_moe_forward(const hfq4_layer *layer, const void *x, hfq_dtype x_
 size_t hfq4_stack_workspace_bytes(int T, int k, int hidden, int inter, int n_experts)
 {
     if (T < 1 || T > 8 || k < 1 || hidden < 1 || inter < 1 || n_experts < 1) return 0;
+    // + the routed stack's logit exchange words [2][E] and logits [T][E]
     return stack_ctl_bytes() + h_bytes(T, k, inter) + 2 * act_bytes(T, hidden) +
-           ((size_t)T * k * 8 + 255) / 256 * 256;
+           ((size_t)T * k * 8 + 255) / 256 * 256 + ((size_t)2 * n_experts * 8 + 255) / 256 * 256 +
+           ((size_t)T * n_experts * 4 + 255) / 256 * 256;
 }
 
 int hfq4_stack_launches(int n_layers, int T, int k, int hidden, int inter)
@@ -397,6 +399,70 @@ hfq_status hfq4_moe_decode_stack(const hfq4_layer *layers, int n_layers, const f
         float *y = y_all ? y_all + (size_t)l * T * H : nullptr;
         st = launch_layer(layers[l], cur, HFQ_BF16, T, idx, wts, k, y, nullptr, h, cur, next,
                           static_cast<unsigned *>(workspace), s);
+        if (st) return st;
+        cur = next;
+    }
+    return ok();
+}
+
+hfq_status hfq4_moe_decode_stack_routed(const hfq4_layer *layers, int n_layers, const void *router,
+                                        hfq_dtype router_dtype, int k, const void *x0, int T, void *x_out,
+                                        float *y_all, int32_t *idx_all, float *wts_all, float *logits_all,
+                                        void *workspace, size_t ws_bytes, void *stream)
+{
+    if (!layers || n_layers < 1 || n_layers > HFQ_MAX_STACK_LAYERS)
+        return fail(HFQ_ERR_ARG, "n_layers=%d not in [1, %d]", n_layers, HFQ_MAX_STACK_LAYERS);
+    hfq_status st;
+    for (int l = 0; l < n_layers; ++l) {
+        if ((st = check_layer(&layers[l], k))) return st;
+        if (layers[l].hidden != layers[0].hidden || layers[l].inter != layers[0].inter ||
+            layers[l].n_experts != layers[0].n_experts)
+            return fail(HFQ_ERR_ARG, "layer %d has a different shape", l);
+    }
+    if (!router || !x0 || !x_out) return fail(HFQ_ERR_ARG, "null pointer");
+    if (router_dtype != HFQ_F32 && router_dtype != HFQ_BF16) return fail(HFQ_ERR_ARG, "bad router dtype");
+    if (T < 1 || T > 8) return fail(HFQ_ERR_UNSUPPORTED, "decode stack takes T in [1, 8], got %d", T);
+    if ((idx_all == nullptr) != (wts_all == nullptr))
+        return fail(HFQ_ERR_ARG, "idx_all and wts_all go together");
+    if (!aligned16(x0) || !aligned16(x_out) || !aligned16(router) || (y_all && !aligned16(y_all)))
+        return fail(HFQ_ERR_ALIGN, "x0, x_out, router and y_all must be 16-byte aligned");
+    const int H = layers[0].hidden, I = layers[0].inter, E = layers[0].n_experts;
+    size_t need = hfq4_stack_workspace_bytes(T, k, H, I, E);
+    if ((st = check_ws(workspace, ws_bytes, need))) return st;
+    char *ws = static_cast<char *>(workspace) + stack_ctl_bytes();
+    float *h = reinterpret_cast<float *>(ws);
+    ws += h_bytes(T, k, I);
+    uint16_t *xa = reinterpret_cast<uint16_t *>(ws);
+    ws += act_bytes(T, H);
+    uint16_t *xb = reinterpret_cast<uint16_t *>(ws);
+    ws += act_bytes(T, H);
+    ws += ((size_t)T * k * 8 + 255) / 256 * 256;
+    uint64_t *lbuf = reinterpret_cast<uint64_t *>(ws);
+    ws += ((size_t)2 * E * 8 + 255) / 256 * 256;
+    float *lscratch = reinterpret_cast<float *>(ws);
+    cudaStream_t s = (cudaStream_t)stream;
+    unsigned *ctl = static_cast<unsigned *>(workspace);
+    const bool bf16 = router_dtype == HFQ_BF16;
+    if (T == 1 && bf16 && stack_supported(T, H, I, k, num_sms_fwd())) {
+        // the router fused into the one-token kernel
+        st = decode1_launch(layers, n_layers, nullptr, nullptr, nullptr, x0, false, k,
+                            static_cast<uint16_t *>(x_out), xa, h, y_all, nullptr, idx_all, wts_all, ctl,
+                            option_wait_timeout_ns(), option_take_extra_arrivals(), s,
+                            static_cast<const uint16_t *>(router), lbuf, logits_all);
+        if (st != HFQ_ERR_UNSUPPORTED) return st ? st : ok();
+    }
+    // otherwise layer by layer: the router GEMV, then the layer on its logits
+    const size_t rstride = (size_t)E * H * (bf16 ? 2 : 4);
+    const void *cur = x0;
+    for (int l = 0; l < n_layers; ++l) {
+        float *lg = logits_all ? logits_all + (size_t)l * T * E : lscratch;
+        if ((st = launch_router(cur, true, static_cast<const char *>(router) + l * rstride, bf16, T, E, H, lg, s)))
+            return st;
+        void *next = (l == n_layers - 1) ? x_out : (void *)(l & 1 ? xb : xa);
+        st = hfq4_moe_decode_stack(&layers[l], 1, lg, k, cur, T, next, y_all ? y_all + (size_t)l * T * H : nullptr,
+                                   idx_all ? idx_all + (size_t)l * T * k : nullptr,
+                                   wts_all ? wts_all + (size_t)l * T * k : nullptr, HFQ_PATH_AUTO, workspace,
+                                   ws_bytes, stream);
         if (st) return st;
         cur = next;
     }

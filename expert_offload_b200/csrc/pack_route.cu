@@ -228,11 +228,66 @@ int num_sms()
 }
 
 }  // namespace
+
+// Router GEMV: logits[t][e] = sum_h x[t][h] * Wr[e][h] with f32 accumulation
+// in a fixed order: lane l takes the 8-value chunks h0 = 8 l + 256 i in turn,
+// each chunk's products in order, then a fixed warp tree; the one-token
+// persistent kernel's fused router uses the same order (same bits).  One warp
+// per (token, expert), consecutive lanes on consecutive chunks.
+__global__ void router_kernel(const void *__restrict__ x, int x_bf16, const void *__restrict__ wr, int wr_bf16,
+                              int T, int E, int H, float *__restrict__ logits)
+{
+    const int wg = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
+    if (wg >= T * E) return;
+    const int t = wg / E, e = wg - t * E;
+    float acc = 0.0f;
+    for (int h0 = 8 * lane; h0 < H; h0 += 256) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const size_t xi = (size_t)t * H + h0 + i, wi = (size_t)e * H + h0 + i;
+            const float xv = x_bf16 ? bf16_bits_to_float(static_cast<const uint16_t *>(x)[xi])
+                                    : static_cast<const float *>(x)[xi];
+            const float wv = wr_bf16 ? bf16_bits_to_float(static_cast<const uint16_t *>(wr)[wi])
+                                     : static_cast<const float *>(wr)[wi];
+            acc = fmaf(xv, wv, acc);
+        }
+    }
+    acc = warp_sum(acc);
+    if (lane == 0) logits[(size_t)t * E + e] = acc;
+}
+
+hfq_status launch_router(const void *x, bool x_bf16, const void *wr, bool wr_bf16, int T, int E, int H,
+                         float *logits, cudaStream_t s)
+{
+    const size_t warps = (size_t)T * E;
+    router_kernel<<<(unsigned)((warps + 7) / 8), 256, 0, s>>>(x, x_bf16 ? 1 : 0, wr, wr_bf16 ? 1 : 0, T, E, H,
+                                                              logits);
+    cudaError_t err = cudaGetLastError();
+    if (err != cudaSuccess) return fail(HFQ_ERR_CUDA, "router launch: %s", cudaGetErrorString(err));
+    return HFQ_OK;
+}
+
 }  // namespace hfq
 
 using namespace hfq;
 
 extern "C" {
+
+hfq_status moe_router_logits(const void *x, hfq_dtype x_dtype, int T, int hidden, const void *router,
+                             hfq_dtype router_dtype, int n_experts, float *logits, void *stream)
+{
+    if (!x || !router || !logits) return fail(HFQ_ERR_ARG, "moe_router_logits: null pointer");
+    if ((x_dtype != HFQ_F32 && x_dtype != HFQ_BF16) || (router_dtype != HFQ_F32 && router_dtype != HFQ_BF16))
+        return fail(HFQ_ERR_ARG, "moe_router_logits: bad dtype");
+    if (T < 1 || T > 65536 || hidden < 8 || hidden % 8 || n_experts < 1 || n_experts > HFQ_MAX_EXPERTS)
+        return fail(HFQ_ERR_UNSUPPORTED, "moe_router_logits: T=%d hidden=%d n_experts=%d outside the limits",
+                    T, hidden, n_experts);
+    if (((uintptr_t)x & 15) || ((uintptr_t)router & 15))
+        return fail(HFQ_ERR_ALIGN, "moe_router_logits: x and router must be 16-byte aligned");
+    const hfq_status st = launch_router(x, x_dtype == HFQ_BF16, router, router_dtype == HFQ_BF16, T, n_experts,
+                                        hidden, logits, (cudaStream_t)stream);
+    return st ? st : ok();
+}
 
 hfq_status hfq4_pack_experts_device(const float *gate, const float *up, const float *down,
                                     int n_experts, int hidden, int inter, void *out,

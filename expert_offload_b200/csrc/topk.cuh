@@ -127,7 +127,9 @@ __device__ __forceinline__ void warp_route(const float *row, int E, int k, int &
 // round), so the merge's lowest-candidate tie rule is the lowest expert, and
 // the selection and weights are those of warp_route.  E % (kWarps * 32) == 0
 // or E / kWarps <= 32; k <= 16.  Warp 0 lane j < k returns (e_j, w_j).
-template <int kWarps>
+// kShared: `row` is in shared memory (plain loads instead of the read-only
+// global path).
+template <int kWarps, bool kShared = false>
 __device__ __forceinline__ void cta_route(const float *row, int E, int k, uint32_t *cand_key, int *cand_e,
                                           int &my_e, float &my_w)
 {
@@ -141,7 +143,7 @@ __device__ __forceinline__ void cta_route(const float *row, int E, int k, uint32
             cand_e[warp * k + j] = e;
         }
     };
-    auto key_g = [&](int c) { return order_key(__ldg(row + base + c)); };
+    auto key_g = [&](int c) { return order_key(kShared ? row[base + c] : __ldg(row + base + c)); };
     auto id_g = [&](int c) { return base + c; };
     if (C <= 32) warp_topk_core<1>(key_g, id_g, C, k, e_, w_, keep);
     else warp_topk_core<2>(key_g, id_g, C, k, e_, w_, keep);
@@ -158,40 +160,3 @@ __device__ __forceinline__ void cta_route(const float *row, int E, int k, uint32
 
 }  // namespace hfq
 
-namespace hfq {
-
-// cta_route with the merge done by every warp: after the block barrier each
-// warp merges the kWarps * k candidates itself, so lane j < k of EVERY warp
-// returns (e_j, w_j) and no second barrier is needed before a warp acts on its
-// slots.  `before_barrier` runs on every thread just before the barrier (work
-// that the merged result's users need complete, such as waiting for an async
-// copy this thread issued).
-template <int kWarps, class F>
-__device__ __forceinline__ void cta_route_all(const float *row, int E, int k, uint32_t *cand_key, int *cand_e,
-                                              int &my_e, float &my_w, F &&before_barrier)
-{
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int C = E / kWarps, base = warp * C;
-    int e_ = -1;
-    float w_ = 0.0f;
-    auto keep = [&](int j, int e, uint32_t m) {
-        if (lane == 0) {
-            cand_key[warp * k + j] = m;
-            cand_e[warp * k + j] = e;
-        }
-    };
-    auto key_g = [&](int c) { return order_key(__ldg(row + base + c)); };
-    auto id_g = [&](int c) { return base + c; };
-    if (C <= 32) warp_topk_core<1>(key_g, id_g, C, k, e_, w_, keep);
-    else warp_topk_core<2>(key_g, id_g, C, k, e_, w_, keep);
-    before_barrier();
-    __syncthreads();
-    const int n = kWarps * k;
-    auto key_s = [&](int c) { return cand_key[c]; };
-    auto id_s = [&](int c) { return cand_e[c]; };
-    auto none = [](int, int, uint32_t) {};
-    if (n <= 64) warp_topk_core<2>(key_s, id_s, n, k, my_e, my_w, none);
-    else warp_topk_core<4>(key_s, id_s, n, k, my_e, my_w, none);
-}
-
-}  // namespace hfq

@@ -21,6 +21,8 @@
  *           registered with the CUDA runtime, 2 MiB pages when available.
  *   [WMMA]  gfx1151 engine README, Windows section: a self-written matrix-
  *           core GEMM for prefill (prior art for the tensor-core path).
+ *   [CACHE] Strata user report, section "model and engine": hot experts in a
+ *           VRAM cache in front of the pinned host arena.
  *
  * Conventions shared by every entry point:
  *   - Weights: w = zero + scale * q with q in [0, 15].  Block layout: f32
@@ -143,6 +145,24 @@ hfq_status moe_route(const float *logits, int T, int E, int k, int32_t *idx, flo
                      size_t ws_bytes, void *stream);
 
 /*
+ * Router logits (device): logits[t][e] = sum_c x[t][c] * Wr[e][c], the plain
+ * linear map of each token's hidden state that picks its layer's experts
+ * (hipfire offload explainer, opening section: each token's router selects 8
+ * of the layer's experts; no bias).
+ *   x:      [T][hidden] in x_dtype (f32 or bf16), 16-byte aligned.
+ *   router: Wr [n_experts][hidden] in router_dtype (f32 or bf16), 16-byte
+ *           aligned.  hidden must be a multiple of 8.
+ *   logits: f32 [T][n_experts] out.
+ * Summation order (fixed, so every call and the fused router in the decode
+ * stack give the same bits): each of 32 lanes sums its 8-column chunks
+ * c0 = 8*lane + 256*i in order, then the 32 lane sums are added by a
+ * butterfly (xor 16, 8, 4, 2, 1).  Returns HFQ_ERR_ARG / HFQ_ERR_ALIGN on bad
+ * arguments, HFQ_ERR_CUDA on a launch error.
+ */
+hfq_status moe_router_logits(const void *x, hfq_dtype x_dtype, int T, int hidden, const void *router,
+                             hfq_dtype router_dtype, int n_experts, float *logits, void *stream);
+
+/*
  * One MoE layer's experts [TABLE][PCIE].
  *   expert_ptr: DEVICE array [n_experts] of base addresses of the packed
  *               experts, each 16-byte aligned; an address may be HBM or a
@@ -217,6 +237,27 @@ hfq_status hfq4_moe_decode_stack(const hfq4_layer *layers, int n_layers, const f
                                  int k, const void *x0, int T, void *x_out, float *y_all,
                                  int32_t *idx_all, float *wts_all, int path, void *workspace,
                                  size_t ws_bytes, void *stream);
+
+/*
+ * The same decode stack with each layer's router in the loop: layer l's
+ * logits are computed from x_l by moe_router_logits' arithmetic (same bits)
+ * instead of being read from memory, so the residual stream decides the
+ * routing as in the model.
+ *   router:  Wr [n_layers][E][H] in router_dtype (f32 or bf16, device,
+ *            16-byte aligned).
+ *   logits_all: optional f32 [n_layers][T][E] out: every layer's logits.
+ *   The other arguments as for hfq4_moe_decode_stack (path AUTO).  With
+ *   T = 1, a bf16 router and a shape the persistent kernel takes, the whole
+ *   stack, routers included, is one launch: every CTA computes a share of
+ *   the logits and the shares are exchanged through the workspace.
+ *   Otherwise each layer is a router launch followed by a one-layer stack.
+ *   workspace: hfq4_stack_workspace_bytes(T, k, H, I, E) bytes.
+ */
+hfq_status hfq4_moe_decode_stack_routed(const hfq4_layer *layers, int n_layers, const void *router,
+                                        hfq_dtype router_dtype, int k, const void *x0, int T,
+                                        void *x_out, float *y_all, int32_t *idx_all, float *wts_all,
+                                        float *logits_all, void *workspace, size_t ws_bytes,
+                                        void *stream);
 
 /*
  * Allocation-free variant of hfq4_moe_forward.  The pages have no counterpart:
@@ -332,6 +373,56 @@ hfq_status hfq_placement_build(int L, int E, size_t expert_bytes, const uint32_t
 hfq_status hfq_placement_pointers(int L, int E, size_t expert_bytes, const uint8_t *loc,
                                   const int64_t *slot, const void *hbm_base,
                                   const void *host_dev_base, uint64_t *out);
+
+/*
+ * Expert cache over host-mapped experts [CACHE][PCIE] (host; copies and table
+ * writes asynchronous on `stream`).
+ *
+ * Keeps up to `slots` experts of each layer in HBM slots (`slot_mem`, caller
+ * device memory of L * slots * expert_bytes bytes) and maintains the layers'
+ * pointer tables `table_dev` (caller device memory [L][E] u64: the
+ * expert_ptr the kernels read) and, if given, location tables `loc_dev`
+ * ([L][E] u8: the expert_loc they read): an entry names the expert's slot
+ * while it is cached (location 0) and its home otherwise.  home, host_src and
+ * home_loc are host arrays [L][E]: the address the kernels read when the
+ * expert is not cached (HBM, or the device alias of a host-mapped expert),
+ * its pinned host address when it lives in host memory (copy source; 0 for
+ * experts resident in HBM, which are never cached), and 1 for host experts.
+ * table_dev = NULL keeps the bookkeeping only (no device work; policy tests).
+ * The library allocates a small host object and a pinned staging buffer of
+ * 18 E bytes; hfq_cache_destroy frees them.
+ *
+ * hfq_cache_observe: the n expert ids (host array, [0, E)) one step selected
+ * in `layer`.  Each distinct selected expert counts as a hit when the kernels
+ * read it from HBM (resident or cached) and as a miss otherwise; its selection
+ * frequency grows by one (all of the layer's frequencies are halved every 256
+ * observations of the layer).  Missed experts are then admitted, most
+ * frequent first (ties to the lower id), up to max_admit of them: into a free
+ * slot, or in place of the least frequent cached expert not selected in this
+ * call when the newcomer is more frequent.  max_admit = -1 admits every
+ * missed expert whatever the frequencies (copy-engine staging before use, as
+ * long as the slots hold them).  The call first synchronises `stream` (no
+ * earlier write of this cache is pending), then enqueues on it: the layer's
+ * tables with evicted experts back home, the copies of the admitted experts
+ * from pinned host memory into their slots (cudaMemcpyAsync: the copy engine),
+ * then the tables naming the admitted experts' slots.  Kernels launched later
+ * on `stream` read the new tables; none may run on another stream meanwhile.
+ * [CACHE] Strata report, "model and engine": a VRAM cache of hot experts in
+ * front of the pinned host arena, refilled from it.
+ */
+typedef struct hfq_cache hfq_cache;
+hfq_status hfq_cache_create(int L, int E, size_t expert_bytes, int slots, const uint64_t *home,
+                            const uint64_t *host_src, const uint8_t *home_loc, void *slot_mem,
+                            size_t slot_bytes, uint64_t *table_dev, uint8_t *loc_dev, void *stream,
+                            hfq_cache **out);
+hfq_status hfq_cache_observe(hfq_cache *cache, int layer, const int32_t *ids, int n, int max_admit,
+                             void *stream);
+/* Slot of an expert (-1: not cached). */
+hfq_status hfq_cache_slot_of(const hfq_cache *cache, int layer, int expert, int *slot);
+/* Counters since creation (any pointer may be NULL). */
+hfq_status hfq_cache_stats(const hfq_cache *cache, uint64_t *hits, uint64_t *misses,
+                           uint64_t *admitted, uint64_t *evicted);
+hfq_status hfq_cache_destroy(hfq_cache *cache);
 
 /*
  * Read-bandwidth probe: a streaming kernel that reads `bytes` from `src`

@@ -17,6 +17,27 @@ from __future__ import annotations
 import numpy as np
 
 
+def router_logits(x: np.ndarray, wr: np.ndarray) -> np.ndarray:
+    """Router logits [T, E] = x Wr^T in fp64: x [T, H] activation values, Wr
+    [E, H] router weights (hipfire offload explainer, opening section: each
+    token's router picks its layer's experts; the router is the plain linear
+    map of the token's hidden state, no bias)."""
+    x = np.asarray(x, dtype=np.float64)
+    wr = np.asarray(wr, dtype=np.float64)
+    return x @ wr.T
+
+
+def near_ties(logits: np.ndarray, k: int, margin) -> np.ndarray:
+    """bool [T]: rows whose k-th and (k+1)-th largest logits lie within
+    `margin` (scalar or [T]) of each other, where two correct computations of
+    the logits (different rounding) may select different experts."""
+    l = np.asarray(logits, dtype=np.float64)
+    if l.shape[1] <= k:
+        return np.zeros(l.shape[0], dtype=bool)
+    s = -np.sort(-l, axis=1)
+    return (s[:, k - 1] - s[:, k]) <= np.asarray(margin, dtype=np.float64)
+
+
 def softmax(logits: np.ndarray) -> np.ndarray:
     """Row-wise softmax in fp64 with the row maximum subtracted first."""
     l = np.asarray(logits, dtype=np.float64)

@@ -24,10 +24,13 @@ def eo():
     return expert_offload_b200
 
 
-@pytest.fixture(scope="module")
-def offload_model(eo):
+@pytest.fixture(scope="module", params=[False, True], ids=["4k_pages", "2m_pages"])
+def offload_model(eo, request):
     """Layers 0..2 of the 512-expert model; layer 0 in HBM, layers 1-2 on the
-    host except their 51 hottest experts (by calibration counts)."""
+    host except their 51 hottest experts (by calibration counts).  The host
+    arena is made both ways: pinned 4 KiB pages (cudaHostAlloc) and 2 MiB
+    transparent huge pages asked for with madvise, then registered (the
+    Strata report, pitfall 7)."""
     from expert_offload_b200.model import ExpertStore
     w = W.WORKLOADS[5]
     L, E = 3, w.experts
@@ -38,7 +41,8 @@ def offload_model(eo):
     np.testing.assert_array_equal(loc, ref.loc)
     np.testing.assert_array_equal(slot, ref.slot)
     assert int(loc.sum()) == 2 * (E - 51)
-    store = ExpertStore(torch, L, E, w.hidden, w.inter, device_fill(torch, w), loc=loc, slot=slot)
+    store = ExpertStore(torch, L, E, w.hidden, w.inter, device_fill(torch, w), loc=loc, slot=slot,
+                        hugepage=request.param)
     yield w, store, loc
     store.close()
 

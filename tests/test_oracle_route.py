@@ -106,3 +106,22 @@ def test_planted_unnormalised_weights_are_caught():
     p = route.softmax(l)
     raw = np.take_along_axis(p, idx.astype(np.int64), axis=1)
     assert not np.allclose(raw.sum(axis=1), 1.0)     # the renormalisation is load-bearing
+
+
+def test_router_logits_hand_case():
+    """x = [[1, 2], [-1, 0.5]], Wr rows [1, 0], [0.5, -1], [0.25, 0.25]:
+    logits row 0 = [1, 0.5 - 2, 0.25 + 0.5] = [1, -1.5, 0.75],
+    row 1 = [-1, -0.5 - 0.5, -0.25 + 0.125] = [-1, -1, -0.125]."""
+    from oracle.route import router_logits
+    x = np.array([[1.0, 2.0], [-1.0, 0.5]])
+    wr = np.array([[1.0, 0.0], [0.5, -1.0], [0.25, 0.25]])
+    np.testing.assert_array_equal(router_logits(x, wr), [[1.0, -1.5, 0.75], [-1.0, -1.0, -0.125]])
+    idx, _ = route.route(router_logits(x, wr), 2)
+    np.testing.assert_array_equal(idx, [[0, 2], [2, 0]])   # row 1: tie of -1 to the lower index
+
+
+def test_near_ties_flags_the_boundary():
+    from oracle.route import near_ties
+    l = np.array([[3.0, 1.0, 1.0 + 1e-9, 0.0], [3.0, 2.0, 1.0, 0.0]])
+    np.testing.assert_array_equal(near_ties(l, 2, 1e-6), [True, False])
+    np.testing.assert_array_equal(near_ties(l, 4, 1e-6), [False, False])
