@@ -261,8 +261,9 @@ class StackTimer:
     """CUDA graphs of one stack launch per token group, replayed back to back
     on one stream with an event after each launch."""
 
-    def __init__(self, torch, eo, layers, inp, k, H, I, E, path=0):
+    def __init__(self, torch, eo, layers, inp, k, H, I, E, path=0, router=None):
         self.torch, self.eo, self.inp, self.k = torch, eo, inp, k
+        self.router = router
         T, G = inp.T, inp.G
         self.layers = layers
         self.arr = eo.layer_array(layers)
@@ -294,6 +295,12 @@ class StackTimer:
             self.launch_mode = "direct launch"
 
     def step(self, g):
+        if self.router is not None:
+            self.eo.hfq4_moe_decode_stack_routed(self.layers, self.router, self.eo.HFQ_BF16, self.k,
+                                                 self.inp.d_x[g], self.inp.T, self.x_out[g],
+                                                 self.ws, stream=self.stream,
+                                                 _layer_array=self.arr)
+            return
         self.eo.hfq4_moe_decode_stack(self.layers, self.inp.d_logits[g], self.k, self.inp.d_x[g],
                                       self.inp.T, self.x_out[g], self.ws, path=self.path,
                                       stream=self.stream, _layer_array=self.arr)
@@ -507,6 +514,44 @@ TRAFFIC_SOURCE = None
 
 
 # --------------------------------------------------------- the other configs
+
+def run_routed(args, K, W_):
+    """The decode stack with each layer's router in the loop (bf16 Wr, one
+    launch per token): the logits come from the residual stream, so the
+    experts a step reads are known only inside the launch; with one token
+    every layer reads exactly k distinct experts plus its router matrix."""
+    import numpy as np
+    import torch
+
+    import expert_offload_b200 as eo
+    import synth
+    from expert_offload_b200.model import ExpertStore
+    from synth import workloads as W
+
+    w = W.WORKLOADS[2]
+    L, H, I, E, k, T = w.layers, w.hidden, w.inter, w.experts, w.top_k, 1
+    eb = eo.hfq4_expert_bytes(H, I)
+    store = ExpertStore(torch, L, E, H, I, fill_for(torch, synth, W, w))
+    wr = np.stack([W.router_weights(w, l) for l in range(L)])
+    router = torch.from_numpy(synth.to_bf16_bits(wr).view(np.int16)).cuda()
+    inp = StackInputs(torch, W, w, 1, T, args.distinct_tokens)      # x0 per token; logits unused
+    timer = StackTimer(torch, eo, store.layers, inp, k, H, I, E, router=router)
+    total_ms, per_launch, clocks = timer.run(K, W_)
+    launches = eo.hfq4_stack_launches(L, T, k, H, I)
+    bytes_step = L * (k * eb + E * H * 2)
+    peak, peak_kind = peaks()
+    roof = hbm_roofline(bytes_step, sum(per_launch) / K, peak, peak_kind, None,
+                        kernel_name(T, launches) + ", router fused")
+    res = {"decode_routed": sub_result(
+        T, K, total_ms, per_launch, clocks, roof, launches,
+        {"workload": w.name + ", bf16 router in the loop",
+         "bytes_per_step": "L * (k distinct experts + the E x H bf16 router matrix)"})}
+    timer.close()
+    store.close()
+    del store, timer, router
+    torch.cuda.empty_cache()
+    return res
+
 
 def run_verify_suite(args, K, W_):
     """48 x 512 experts, skewed routing, T = 1, 2, 5, 8 (one model, four runs)."""
@@ -1073,6 +1118,7 @@ def main():
         K = max(5, min(args.steps, 50))
         W_ = max(3, min(args.warmup, 10))
         subs = {}
+        subs.update(run_routed(args, K, W_))
         subs.update(run_verify_suite(args, K, W_))
         subs.update(run_offload_suite(args, K, W_))
         subs.update(run_prefill(args, [512, 2048, 8192], K, W_))

@@ -52,6 +52,8 @@ constexpr int kGuRows = 4;              // gate/up rows per batched warp reducti
 constexpr int kXLoads = 4;              // 16-byte input loads per thread (H <= 2048)
 constexpr int kHLoads = 8;              // 16-byte h loads per lane and slot (I <= 1024)
 constexpr int kStamps = 32;             // timeline stamps per layer
+constexpr int kMaxRouterRows = 4;       // router rows per CTA: E <= 512 over >= 128 CTAs
+static_assert(kThr == 256, "the router's summation order has 8 groups of 32 partial sums");
 constexpr int kSmemOptin = 232448;      // 227 KB per CTA on sm_100
 
 struct D1Args {
@@ -80,21 +82,27 @@ struct D1Args {
                               // expect a tag nobody writes
     // shared-memory layout, bytes; a slot is [gate span][up span][down span]
     int slot_bytes, up_off, down_off;
-    int xs_off, ptab_off, ltab_off, ysh_off, lsm_off, sh_off;
+    int xs_off, ptab_off, ltab_off, ysh_off, lsm_off, rsm_off, sh_off;
     int ltab_stride;
 };
 
 struct D1Shared {
     uint64_t gu_bar[kMaxK];           // gate + up span of slot j landed
     uint64_t d_bar[kMaxK];            // down span of slot j landed
+    uint64_t r_bar;                   // this CTA's router rows of a layer landed (one phase per layer)
+    int r_issued;                     // router row copies issued
+    float rpart[kMaxRouterRows * kW];     // router: the warps' partial sums of each row
     const uint8_t *base[kMaxK];       // expert of slot j
     float w[kMaxK];                   // routing weight of slot j
     unsigned hostmask;                // slots whose expert is in host memory
     int abort;
     int last_cta;
     int armed;                        // layers whose slot barriers were armed
-    uint32_t cand_key[kW * kMaxK];    // routing: each warp's top k of its experts
-    int cand_e[kW * kMaxK];
+    alignas(16) uint64_t rkey[HFQ_MAX_EXPERTS];   // routing: every expert's key
+    alignas(16) uint64_t rcand[8 * kMaxK];        // the k best of each group of 64
+    uint64_t rsel[kMaxK];             // the k best, by slot
+    uint32_t rwmax[kW];               // routing (k <= 8): each warp's largest key
+    int rn;                           // routing (k <= 8): experts at or above the bound
 };
 
 // Exchange tag of layer l (< 64) in launch `epoch`: never 0 (a fresh or
@@ -232,20 +240,36 @@ __global__ void __launch_bounds__(kThr, 1) decode1_kernel(const __grid_constant_
     uint8_t *ltab = smem + a.ltab_off;                                // [2][ltab_stride]
     float *ysh = reinterpret_cast<float *>(smem + a.ysh_off);        // [kW][kMaxDRows]
     float *lsm = reinterpret_cast<float *>(smem + a.lsm_off);        // [E] logits (router)
+    uint16_t *rsm = reinterpret_cast<uint16_t *>(smem + a.rsm_off);  // [E/G rows][H] this CTA's Wr rows
     D1Shared &sh = *reinterpret_cast<D1Shared *>(smem + a.sh_off);
     const WaitCtx wc{a.ctl, a.timeout_ns, &sh.abort};
     const uint32_t epoch = *(volatile const unsigned *)(a.ctl + kCtlEpoch);
     const uint32_t sig = xch_signature(k, Ip, H, a.L, a.router ? E : 0);
     const bool reset = *(volatile const unsigned *)(a.ctl + kCtlSig) != sig;
+    // router: CTA c computes the logits of experts [r_lo, r_hi); their Wr rows
+    // are one contiguous span, copied into rsm a layer ahead
+    const bool route_in_kernel = a.router && !a.idx_in;
+    const int r_lo = (int)((long long)c * E / G), r_hi = (int)((long long)(c + 1) * E / G);
+    const uint32_t r_len = route_in_kernel ? (uint32_t)((r_hi - r_lo) * H * 2) : 0u;
+    auto issue_router = [&](int l) {       // thread 0
+        if (r_len) {
+            mbar_arrive_expect_tx(&sh.r_bar, r_len);
+            bulk_g2s_hint(rsm, a.router + ((size_t)l * E + r_lo) * H, r_len, &sh.r_bar, l2_evict_first_policy());
+        }
+        sh.r_issued = l + 1;
+    };
 
     if (tid == 0) {
         for (int j = 0; j < kMaxK; ++j) {
             mbar_init(&sh.gu_bar[j], 1);
             mbar_init(&sh.d_bar[j], 1);
         }
+        mbar_init(&sh.r_bar, 1);
         sh.abort = 0;
         sh.armed = 0;
+        sh.r_issued = 0;
         fence_mbar_init();
+        if (route_in_kernel && a.L > 0) issue_router(0);
     }
     for (int i = H + tid; i < Hp; i += kThr) xs[xp4(i)] = 0.0f;   // padding, never rewritten
     if (warp == 0) fetch_table(a, 0, ptab, ltab);
@@ -330,27 +354,48 @@ __global__ void __launch_bounds__(kThr, 1) decode1_kernel(const __grid_constant_
         if (__syncthreads_or(sh.abort)) break;
         stamp(a, l, 4);
         // ---------------------------------------------- 1a'. router (optional)
-        // logits = Wr_l x_l: CTA c computes experts [c E / G, (c + 1) E / G),
-        // one warp each (the order of moe_router_logits, same bits), writes
-        // them as tagged words, and every CTA polls all E of them into lsm
-        if (a.router && !a.idx_in) {
-            const int r_lo = (int)((long long)c * E / G), r_hi = (int)((long long)(c + 1) * E / G);
+        // logits = Wr_l x_l for experts [r_lo, r_hi) from this CTA's rows in
+        // rsm, in the summation order of moe_router_logits (same bits):
+        // thread j (warp g = j / 32) sums the 8-column chunks 8 j + 2048 i in
+        // order, each warp sums its 32 partials by a butterfly, and the 8 warp
+        // sums are added as ((0+1)+(2+3))+((4+5)+(6+7)).  The logits go out
+        // as tagged words, and every CTA polls all E of them into lsm.
+        if (route_in_kernel) {
             const uint32_t tag = xch_tag(epoch, l);
-            for (int e = r_lo + warp; e < r_hi; e += kW) {
-                const uint16_t *row = a.router + ((size_t)l * E + e) * H;
+            const bool rok = __all_sync(0xffffffffu, !r_len || wait_mbar_phase(wc, &sh.r_bar, par));
+            if (!rok) sh.abort = 1;
+            const int nr = r_hi - r_lo;
+            for (int r = 0; rok && r < nr; ++r) {
+                const uint16_t *row = rsm + (size_t)r * H;
                 float acc = 0.0f;
-                for (int h0 = 8 * lane; h0 < H; h0 += 256) {
-                    const uint4 v = ld_nc_v4(row + h0);
-                    const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        acc = fmaf(xs[xp4(h0 + 2 * i)], __uint_as_float(w4[i] << 16), acc);
-                        acc = fmaf(xs[xp4(h0 + 2 * i + 1)], __uint_as_float(w4[i] & 0xFFFF0000u), acc);
-                    }
+                for (int h0 = 8 * tid; h0 < H; h0 += 8 * kThr) {
+                    const uint4 v = *reinterpret_cast<const uint4 *>(row + h0);
+                    const float4 xa = *reinterpret_cast<const float4 *>(xs + xp4(h0));
+                    const float4 xb = *reinterpret_cast<const float4 *>(xs + xp4(h0) + 4);
+                    acc = fmaf(xa.x, __uint_as_float(v.x << 16), acc);
+                    acc = fmaf(xa.y, __uint_as_float(v.x & 0xFFFF0000u), acc);
+                    acc = fmaf(xa.z, __uint_as_float(v.y << 16), acc);
+                    acc = fmaf(xa.w, __uint_as_float(v.y & 0xFFFF0000u), acc);
+                    acc = fmaf(xb.x, __uint_as_float(v.z << 16), acc);
+                    acc = fmaf(xb.y, __uint_as_float(v.z & 0xFFFF0000u), acc);
+                    acc = fmaf(xb.z, __uint_as_float(v.w << 16), acc);
+                    acc = fmaf(xb.w, __uint_as_float(v.w & 0xFFFF0000u), acc);
                 }
                 acc = warp_sum(acc);
-                if (lane == 0) st_tagged(a.lbuf + (size_t)(l & 1) * E + e, acc, tag);
+                if (lane == 0) sh.rpart[r * kW + warp] = acc;
             }
+            __syncthreads();
+            if (rok && tid < nr) {
+                const float *q = sh.rpart + tid * kW;
+                const float logit = ((q[0] + q[1]) + (q[2] + q[3])) + ((q[4] + q[5]) + (q[6] + q[7]));
+                st_tagged(a.lbuf + (size_t)(l & 1) * E + r_lo + tid, logit, tag);
+                // out now: without the fence the word reached the other CTAs
+                // microseconds later while they polled
+                __threadfence();
+            }
+            // polling starts once this CTA's logits are out (early pollers
+            // slow the writers down)
+            __syncthreads();
             // poll: thread tid reads logits tid and tid + kThr (E <= 512)
             const uint64_t *lw = a.lbuf + (size_t)(l & 1) * E;
             unsigned pend = (tid < E ? 1u : 0u) | (tid + kThr < E ? 2u : 0u);
@@ -380,6 +425,12 @@ __global__ void __launch_bounds__(kThr, 1) decode1_kernel(const __grid_constant_
                 }
             }
             if (__syncthreads_or(sh.abort)) break;
+            stamp(a, l, 31);
+            // rsm is free again: the next layer's rows travel during this layer
+            if (tid == 0 && l + 1 < n_layers) {
+                fence_proxy_async_smem();
+                issue_router(l + 1);
+            }
             if (a.logits_out && c == 0)
                 for (int e = tid; e < E; e += kThr) a.logits_out[(size_t)l * E + e] = lsm[e];
         }
@@ -387,8 +438,12 @@ __global__ void __launch_bounds__(kThr, 1) decode1_kernel(const __grid_constant_
         int re = -1;
         float rw = 0.0f;
         if (!a.idx_in) {
-            if (a.router) cta_route<kW, true>(lsm, E, k, sh.cand_key, sh.cand_e, re, rw);
-            else cta_route<kW>(a.logits + (size_t)l * E, E, k, sh.cand_key, sh.cand_e, re, rw);
+            const float *row = a.router ? lsm : a.logits + (size_t)l * E;
+            auto logit_of = [&](int e) { return a.router ? row[e] : __ldg(row + e); };
+            if (k <= kW)
+                cta_route_small_k<kThr>(logit_of, E, k, sh.rkey, sh.rwmax, &sh.rn, sh.rsel, re, rw);
+            else
+                cta_route_rank<kThr>(logit_of, E, k, sh.rkey, sh.rcand, sh.rsel, re, rw);
         }
         if (warp == 0) {
             // ------------------------------------------ 1c. issue copies
@@ -694,6 +749,11 @@ __global__ void __launch_bounds__(kThr, 1) decode1_kernel(const __grid_constant_
     }
 
     // no copy may still be writing this CTA's shared memory when it exits
+    if (tid == 0 && r_len && sh.r_issued > 0) {
+        const uint64_t t0 = globaltimer_ns();
+        while (!mbar_try_wait(&sh.r_bar, (uint32_t)(sh.r_issued - 1) & 1u) && !deadline_passed(t0, a.timeout_ns)) {
+        }
+    }
     if (warp == 0) {
         cp_async_wait_all();
         const int armed = sh.armed;
@@ -769,7 +829,8 @@ hfq_status decode1_launch(const hfq4_layer *layers, int L, const float *logits, 
         a.eptr[l] = layers[l].expert_ptr;
         a.eloc[l] = layers[l].expert_loc;
     }
-    if (router && (!lbuf || !aligned16(router) || H % 8)) return HFQ_ERR_UNSUPPORTED;
+    if (router && (!lbuf || !aligned16(router) || H % 8 || (E + G - 1) / G > kMaxRouterRows))
+        return HFQ_ERR_UNSUPPORTED;
     a.logits = logits; a.idx_in = idx_in; a.wts_in = wts_in; a.x0 = x0; a.x_out = x_out;
     a.router = router; a.lbuf = lbuf; a.logits_out = logits_out;
     a.xbuf = reinterpret_cast<uint64_t *>(xbuf); a.h = reinterpret_cast<uint64_t *>(h); a.y = y; a.y_bf16 = y_bf16; a.idx_all = idx_all; a.wts_all = wts_all;
@@ -800,6 +861,9 @@ hfq_status decode1_launch(const hfq4_layer *layers, int L, const float *logits, 
     off += (size_t)kW * kMaxDRows * 4;
     a.lsm_off = (int)off;
     off += router ? up16((size_t)E * 4) : 0;
+    off = up16(off);
+    a.rsm_off = (int)off;
+    off += router ? up16((size_t)((E + G - 1) / G) * H * 2) : 0;
     a.sh_off = (int)up16(off);
     const size_t smem = (size_t)a.sh_off + sizeof(D1Shared);
 

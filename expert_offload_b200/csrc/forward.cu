@@ -336,8 +336,10 @@ hfq_status hfq4_moe_forward(const hfq4_layer *layer, const void *x, hfq_dtype x_
 size_t hfq4_stack_workspace_bytes(int T, int k, int hidden, int inter, int n_experts)
 {
     if (T < 1 || T > 8 || k < 1 || hidden < 1 || inter < 1 || n_experts < 1) return 0;
-    // + the routed stack's logit exchange words [2][E] and logits [T][E]
-    return stack_ctl_bytes() + h_bytes(T, k, inter) + 2 * act_bytes(T, hidden) +
+    // + the routed stack's logit exchange words [2][E], logits [T][E] and its
+    // own pair of residual buffers (its per-layer fallback chains one-layer
+    // stacks, which use the first pair)
+    return stack_ctl_bytes() + h_bytes(T, k, inter) + 4 * act_bytes(T, hidden) +
            ((size_t)T * k * 8 + 255) / 256 * 256 + ((size_t)2 * n_experts * 8 + 255) / 256 * 256 +
            ((size_t)T * n_experts * 4 + 255) / 256 * 256;
 }
@@ -432,14 +434,15 @@ hfq_status hfq4_moe_decode_stack_routed(const hfq4_layer *layers, int n_layers, 
     char *ws = static_cast<char *>(workspace) + stack_ctl_bytes();
     float *h = reinterpret_cast<float *>(ws);
     ws += h_bytes(T, k, I);
-    uint16_t *xa = reinterpret_cast<uint16_t *>(ws);
-    ws += act_bytes(T, H);
-    uint16_t *xb = reinterpret_cast<uint16_t *>(ws);
-    ws += act_bytes(T, H);
+    uint16_t *xa = reinterpret_cast<uint16_t *>(ws);        // with the next buffer: the x exchange
+    ws += 2 * act_bytes(T, H);
     ws += ((size_t)T * k * 8 + 255) / 256 * 256;
     uint64_t *lbuf = reinterpret_cast<uint64_t *>(ws);
     ws += ((size_t)2 * E * 8 + 255) / 256 * 256;
     float *lscratch = reinterpret_cast<float *>(ws);
+    ws += ((size_t)T * E * 4 + 255) / 256 * 256;
+    uint16_t *ra = reinterpret_cast<uint16_t *>(ws);
+    uint16_t *rb = reinterpret_cast<uint16_t *>(ws + act_bytes(T, H));
     cudaStream_t s = (cudaStream_t)stream;
     unsigned *ctl = static_cast<unsigned *>(workspace);
     const bool bf16 = router_dtype == HFQ_BF16;
@@ -458,7 +461,7 @@ hfq_status hfq4_moe_decode_stack_routed(const hfq4_layer *layers, int n_layers, 
         float *lg = logits_all ? logits_all + (size_t)l * T * E : lscratch;
         if ((st = launch_router(cur, true, static_cast<const char *>(router) + l * rstride, bf16, T, E, H, lg, s)))
             return st;
-        void *next = (l == n_layers - 1) ? x_out : (void *)(l & 1 ? xb : xa);
+        void *next = (l == n_layers - 1) ? x_out : (void *)(l & 1 ? rb : ra);
         st = hfq4_moe_decode_stack(&layers[l], 1, lg, k, cur, T, next, y_all ? y_all + (size_t)l * T * H : nullptr,
                                    idx_all ? idx_all + (size_t)l * T * k : nullptr,
                                    wts_all ? wts_all + (size_t)l * T * k : nullptr, HFQ_PATH_AUTO, workspace,

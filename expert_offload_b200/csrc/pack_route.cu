@@ -230,30 +230,38 @@ int num_sms()
 }  // namespace
 
 // Router GEMV: logits[t][e] = sum_h x[t][h] * Wr[e][h] with f32 accumulation
-// in a fixed order: lane l takes the 8-value chunks h0 = 8 l + 256 i in turn,
-// each chunk's products in order, then a fixed warp tree; the one-token
-// persistent kernel's fused router uses the same order (same bits).  One warp
-// per (token, expert), consecutive lanes on consecutive chunks.
+// in a fixed order: 256 partial sums p_j (j = 32 g + lane, g = 0..7), p_j
+// taking the 8-value chunks h0 = 8 j + 2048 i in turn (each chunk's products
+// in order, fmaf); each group g of 32 partials summed by a butterfly over the
+// lanes (xor 16, 8, 4, 2, 1); the 8 group sums added as
+// ((q0 + q1) + (q2 + q3)) + ((q4 + q5) + (q6 + q7)).  The one-token
+// persistent kernel's fused router takes the same steps with its 8 warps as
+// the groups (same bits).  Here one warp per (token, expert) holds the 8
+// groups' partials of its lane.
 __global__ void router_kernel(const void *__restrict__ x, int x_bf16, const void *__restrict__ wr, int wr_bf16,
                               int T, int E, int H, float *__restrict__ logits)
 {
     const int wg = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
     if (wg >= T * E) return;
     const int t = wg / E, e = wg - t * E;
-    float acc = 0.0f;
-    for (int h0 = 8 * lane; h0 < H; h0 += 256) {
+    float q[8];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            const size_t xi = (size_t)t * H + h0 + i, wi = (size_t)e * H + h0 + i;
-            const float xv = x_bf16 ? bf16_bits_to_float(static_cast<const uint16_t *>(x)[xi])
-                                    : static_cast<const float *>(x)[xi];
-            const float wv = wr_bf16 ? bf16_bits_to_float(static_cast<const uint16_t *>(wr)[wi])
-                                     : static_cast<const float *>(wr)[wi];
-            acc = fmaf(xv, wv, acc);
+    for (int g = 0; g < 8; ++g) {
+        float acc = 0.0f;
+        for (int h0 = 8 * (32 * g + lane); h0 < H; h0 += 2048) {
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const size_t xi = (size_t)t * H + h0 + i, wi = (size_t)e * H + h0 + i;
+                const float xv = x_bf16 ? bf16_bits_to_float(static_cast<const uint16_t *>(x)[xi])
+                                        : static_cast<const float *>(x)[xi];
+                const float wv = wr_bf16 ? bf16_bits_to_float(static_cast<const uint16_t *>(wr)[wi])
+                                         : static_cast<const float *>(wr)[wi];
+                acc = fmaf(xv, wv, acc);
+            }
         }
+        q[g] = warp_sum(acc);
     }
-    acc = warp_sum(acc);
-    if (lane == 0) logits[(size_t)t * E + e] = acc;
+    if (lane == 0) logits[(size_t)t * E + e] = ((q[0] + q[1]) + (q[2] + q[3])) + ((q[4] + q[5]) + (q[6] + q[7]));
 }
 
 hfq_status launch_router(const void *x, bool x_bf16, const void *wr, bool wr_bf16, int T, int E, int H,

@@ -1,5 +1,6 @@
-// topk.cuh - routing of one token by one warp: the k largest router logits
-// (ties to the lower expert index) and their softmax over the selected k
+// topk.cuh - routing of one token, by one warp or by a whole CTA: the k
+// largest router logits (ties to the lower expert index) and their softmax
+// over the selected k
 // (hipfire offload explainer, opening section: top-k experts per token,
 // weights renormalised over the chosen ones).
 #pragma once
@@ -120,41 +121,127 @@ __device__ __forceinline__ void warp_route(const float *row, int E, int k, int &
     warp_route_rounds(row, E, k, my_e, my_w, [](int, int) {});
 }
 
-// Routing of one token by all kWarps warps of a CTA: warp w takes the top k
-// of experts [w * E / kWarps, (w + 1) * E / kWarps) into cand_key/cand_e
-// (shared, [kWarps][k]); after a block barrier, warp 0 merges the kWarps * k
-// candidates.  Candidates of equal keys are in expert order (warp, then
-// round), so the merge's lowest-candidate tie rule is the lowest expert, and
-// the selection and weights are those of warp_route.  E % (kWarps * 32) == 0
-// or E / kWarps <= 32; k <= 16.  Warp 0 lane j < k returns (e_j, w_j).
-// kShared: `row` is in shared memory (plain loads instead of the read-only
-// global path).
-template <int kWarps, bool kShared = false>
-__device__ __forceinline__ void cta_route(const float *row, int E, int k, uint32_t *cand_key, int *cand_e,
-                                          int &my_e, float &my_w)
+// Routing of one token by a whole CTA of kThreads threads by ranks (E <=
+// 2 kThreads, k <= 16): every logit gets the 64-bit key
+// (order_key(v) << 32) | (0xFFFFFFFF - e), unique and larger for the better
+// expert (equal logits: the lower index first), and an expert's rank is the
+// number of larger keys.  Step 1 ranks each expert within its group of 64
+// (keys in shared memory, read by broadcast, 0 past E); the k best of each
+// group are the candidates.  Step 2 ranks the candidates among themselves:
+// the k best candidates are the k best experts, the one of rank r taking
+// slot r.  The selection and the weights are those of warp_route: warp 0
+// lane j < k returns e_j and w_j = exp(v_j - v_0) / s, s = sum over i < k of
+// exp(v_i - v_0) added in slot order; other threads return -1.
+// keys: shared [E rounded up to 64], cand: shared [ceil(E / 64) * k rounded
+// up to 8], sel: shared [k]; keys and cand 16-byte aligned.
+template <int kThreads, class LogitOf>
+__device__ __forceinline__ void cta_route_rank(LogitOf &&logit_of, int E, int k, uint64_t *keys, uint64_t *cand,
+                                               uint64_t *sel, int &my_e, float &my_w)
 {
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int C = E / kWarps, base = warp * C;
-    int e_ = -1;
-    float w_ = 0.0f;
-    auto keep = [&](int j, int e, uint32_t m) {
-        if (lane == 0) {
-            cand_key[warp * k + j] = m;
-            cand_e[warp * k + j] = e;
-        }
-    };
-    auto key_g = [&](int c) { return order_key(kShared ? row[base + c] : __ldg(row + base + c)); };
-    auto id_g = [&](int c) { return base + c; };
-    if (C <= 32) warp_topk_core<1>(key_g, id_g, C, k, e_, w_, keep);
-    else warp_topk_core<2>(key_g, id_g, C, k, e_, w_, keep);
+    const int tid = threadIdx.x;
+    const int E64 = (E + 63) & ~63, nc = ((E + 63) >> 6) * k, nc8 = (nc + 7) & ~7;
+    for (int e = tid; e < E64; e += kThreads)
+        keys[e] = e < E ? ((uint64_t)order_key(logit_of(e)) << 32) | (0xFFFFFFFFu - (uint32_t)e) : 0ull;
+    for (int c = tid; c < nc8; c += kThreads) cand[c] = 0ull;      // below every key
     __syncthreads();
+    for (int e = tid; e < E; e += kThreads) {
+        const uint64_t K = keys[e];
+        const ulonglong2 *g = reinterpret_cast<const ulonglong2 *>(keys + (e & ~63));
+        int r = 0;
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+            const ulonglong2 p = g[j];
+            r += (p.x > K ? 1 : 0) + (p.y > K ? 1 : 0);
+        }
+        if (r < k) cand[(e >> 6) * k + r] = K;
+    }
+    __syncthreads();
+    for (int c = tid; c < nc; c += kThreads) {
+        const uint64_t K = cand[c];
+        const ulonglong2 *g = reinterpret_cast<const ulonglong2 *>(cand);
+        int r = 0;
+#pragma unroll 4
+        for (int j = 0; j < nc8 / 2; ++j) {
+            const ulonglong2 p = g[j];
+            r += (p.x > K ? 1 : 0) + (p.y > K ? 1 : 0);
+        }
+        if (K != 0ull && r < k) sel[r] = K;
+    }
+    __syncthreads();
+    my_e = -1;
+    my_w = 0.0f;
+    if (tid < 32) {
+        const float v0 = key_value((uint32_t)(sel[0] >> 32));
+        float s = 0.0f, mine = 0.0f;
+        for (int j = 0; j < k; ++j) {
+            const float ex = __expf(key_value((uint32_t)(sel[j] >> 32)) - v0);
+            s += ex;
+            mine = j == tid ? ex : mine;
+        }
+        if (tid < k) {
+            my_e = (int)(0xFFFFFFFFu - (uint32_t)sel[tid]);
+            my_w = mine / s;
+        }
+    }
+}
+
+// Routing of one token by a whole CTA for k <= kThreads / 32 (E <= 2
+// kThreads): the same selection and weights as cta_route_rank with far less
+// work.  tau = the smallest of the warps' maxima is a lower bound of the
+// k-th largest logit (the kThreads / 32 warp maxima are that many distinct
+// experts), so only experts with key >= tau can be selected; they are
+// gathered (any order) and ranked among themselves by their unique 64-bit
+// keys.  surv: shared [E] keys; wmax: shared [kThreads / 32]; n_surv: a
+// shared counter; sel: shared [k].  Warp 0 lane j < k returns (e_j, w_j).
+template <int kThreads, class LogitOf>
+__device__ __forceinline__ void cta_route_small_k(LogitOf &&logit_of, int E, int k, uint64_t *surv, uint32_t *wmax,
+                                                  int *n_surv, uint64_t *sel, int &my_e, float &my_w)
+{
+    constexpr int kWarps = kThreads / 32;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    uint32_t key[2];
+    uint32_t m = 0u;
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+        const int e = tid + i * kThreads;
+        key[i] = e < E ? order_key(logit_of(e)) : 0u;
+        m = key[i] > m ? key[i] : m;
+    }
+    m = __reduce_max_sync(0xffffffffu, m);
+    if (lane == 0) wmax[warp] = m;
+    if (tid == 0) *n_surv = 0;
+    __syncthreads();
+    uint32_t tau = wmax[0];
+#pragma unroll
+    for (int w = 1; w < kWarps; ++w) tau = wmax[w] < tau ? wmax[w] : tau;
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+        const int e = tid + i * kThreads;
+        if (e < E && key[i] >= tau) surv[atomicAdd(n_surv, 1)] = ((uint64_t)key[i] << 32) | (0xFFFFFFFFu - (uint32_t)e);
+    }
+    __syncthreads();
+    const int n = *n_surv;
+    for (int c = tid; c < n; c += kThreads) {
+        const uint64_t K = surv[c];
+        int r = 0;
+#pragma unroll 4
+        for (int j = 0; j < n; ++j) r += surv[j] > K ? 1 : 0;
+        if (r < k) sel[r] = K;
+    }
+    __syncthreads();
+    my_e = -1;
+    my_w = 0.0f;
     if (warp == 0) {
-        const int n = kWarps * k;
-        auto key_s = [&](int c) { return cand_key[c]; };
-        auto id_s = [&](int c) { return cand_e[c]; };
-        auto none = [](int, int, uint32_t) {};
-        if (n <= 64) warp_topk_core<2>(key_s, id_s, n, k, my_e, my_w, none);
-        else warp_topk_core<4>(key_s, id_s, n, k, my_e, my_w, none);
+        const uint64_t K = lane < k ? sel[lane] : 0ull;
+        const float v = key_value((uint32_t)(K >> 32));
+        const float v0 = __shfl_sync(0xffffffffu, v, 0);
+        const float ex = __expf(v - v0);
+        float s = 0.0f;
+        for (int j = 0; j < k; ++j) s += __shfl_sync(0xffffffffu, ex, j);
+        if (lane < k) {
+            my_e = (int)(0xFFFFFFFFu - (uint32_t)K);
+            my_w = ex / s;
+        }
     }
 }
 

@@ -154,10 +154,13 @@ hfq_status moe_route(const float *logits, int T, int E, int k, int32_t *idx, flo
  *           aligned.  hidden must be a multiple of 8.
  *   logits: f32 [T][n_experts] out.
  * Summation order (fixed, so every call and the fused router in the decode
- * stack give the same bits): each of 32 lanes sums its 8-column chunks
- * c0 = 8*lane + 256*i in order, then the 32 lane sums are added by a
- * butterfly (xor 16, 8, 4, 2, 1).  Returns HFQ_ERR_ARG / HFQ_ERR_ALIGN on bad
- * arguments, HFQ_ERR_CUDA on a launch error.
+ * stack give the same bits): 256 partial sums p_j, j = 32*g + lane
+ * (g = 0..7), each taking the 8-column chunks c0 = 8*j + 2048*i in turn (the
+ * chunk's products in order, fused multiply-add); each group g's 32 partials
+ * added by a butterfly over the lanes (xor 16, 8, 4, 2, 1); the group sums
+ * added as ((q0+q1)+(q2+q3))+((q4+q5)+(q6+q7)).  Returns HFQ_ERR_ARG /
+ * HFQ_ERR_ALIGN on bad arguments, HFQ_ERR_UNSUPPORTED beyond the limits,
+ * HFQ_ERR_CUDA on a launch error.
  */
 hfq_status moe_router_logits(const void *x, hfq_dtype x_dtype, int T, int hidden, const void *router,
                              hfq_dtype router_dtype, int n_experts, float *logits, void *stream);

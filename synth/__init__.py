@@ -1,9 +1,9 @@
 """Seeded synthetic inputs for the routed-expert HFQ4 MoE layer.
 
 This module is the one piece that both the oracle side and the CUDA side
-consume.  It holds no step of the MoE method (no quantisation, routing,
-expert FFN or combine): it only produces the f32 weights, activations and
-router logits that the workloads are defined on, from counter-based random
+consume.  It holds no step of the MoE method (no quantisation, router GEMV,
+routing, expert FFN or combine): it only produces the f32 weights,
+activations, router weights and logits of the workloads, from counter-based random
 numbers (Philox4x32-10, see ``synth_philox.h``) whose bits are identical on
 the host (``libsynth_host.so``) and on the GPU (``libsynth_dev.so``).
 

@@ -44,7 +44,7 @@ class Workload:
     top_k: int
     tokens: tuple          # token counts the workload is run at
     act_dtype: str         # "f32" or "bf16"
-    logits: str            # "router" | "normal" | "skewed" | "zipf"
+    logits: str            # "normal" | "skewed" | "zipf"
     n_hot: int = 0
     extra: dict = field(default_factory=dict)
 
@@ -54,7 +54,7 @@ class Workload:
 
 
 WORKLOADS = {
-    1: Workload(1, "tiny moe layer h256 i128 e16 top4 t8", 1, 256, 128, 16, 4, (8,), "f32", "router"),
+    1: Workload(1, "tiny moe layer h256 i128 e16 top4 t8", 1, 256, 128, 16, 4, (8,), "f32", "normal"),
     2: Workload(2, "decode stack l40 h2048 i512 e256 top8 t1", 40, 2048, 512, 256, 8, (1,), "bf16",
                 "normal"),
     3: Workload(3, "verify stack l48 h2048 i512 e512 top8 t1/2/5/8 skewed", 48, 2048, 512, 512, 8,
@@ -98,18 +98,9 @@ def router_weights(w: Workload, layer: int = 0) -> np.ndarray:
     return normal(w.seed, STREAM_ROUTER, layer, 0, w.experts, w.hidden, ROUTER_SIGMA)
 
 
-def _has_boundary_tie(logits: np.ndarray, k: int) -> bool:
-    s = -np.sort(-logits.astype(np.float64), axis=1)
-    return bool(np.any(s[:, k - 1] == s[:, k])) if logits.shape[1] > k else False
-
-
 def logits(w: Workload, layer: int, token0: int, T: int) -> np.ndarray:
     """Router logits f32 [T, E] for tokens token0.. at one layer."""
-    if w.logits == "router":
-        x = activations_f32(w, token0, T).astype(np.float64)
-        wr = router_weights(w, layer).astype(np.float64)
-        out = (x @ wr.T).astype(np.float32)
-    elif w.logits == "normal":
+    if w.logits == "normal":
         out = normal_fine(w.seed, STREAM_LOGIT, layer, token0, T, w.experts, 1.0)
     elif w.logits == "skewed":
         beta = skew_beta(w)
@@ -119,11 +110,7 @@ def logits(w: Workload, layer: int, token0: int, T: int) -> np.ndarray:
         out = zipf_logits(w, layer, token0, T)
     else:
         raise ValueError(w.logits)
-    # The tiny workload's seed is checked for ties at the selection boundary
-    # (its recipe excludes them); elsewhere exact ties are merely rare and both
-    # sides break them towards the lower expert index.
-    if w.logits == "router" and _has_boundary_tie(out, w.top_k):
-        raise ValueError(f"seed {w.seed:#x} gives a logit tie at the top-{w.top_k} boundary")
+    # exact ties are rare; both sides break them towards the lower expert index
     return out
 
 
