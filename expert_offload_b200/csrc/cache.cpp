@@ -31,9 +31,12 @@ struct hfq_cache {
     std::vector<int> owner;                // [L][slots]: expert, or -1
     std::vector<float> freq;               // [L][E] selection frequency
     std::vector<uint32_t> nobs;            // [L] observations
-    // pinned staging of one layer's tables: [2][E] pointers, [2][E] locations
+    // pinned staging of the tables: [L][2][E] pointers, [L][2][E] locations,
+    // and per layer an event after the last copy that read its staging
     uint64_t *stage_ptr = nullptr;
     uint8_t *stage_loc = nullptr;
+    std::vector<cudaEvent_t> staged;       // [L]
+    std::vector<char> staged_live;         // [L]: the event was recorded
     uint64_t hits = 0, misses = 0, admitted = 0, evicted = 0;
 };
 
@@ -54,12 +57,12 @@ uint8_t loc_entry(const hfq_cache *c, int l, int e)
     return c->slot_of[i] >= 0 ? 0 : c->home_loc[i];
 }
 
-// Layer l's tables (as the bookkeeping says now) into staging buffer `b`, then
-// to the device.
+// Layer l's tables (as the bookkeeping says now) into its staging buffer `b`,
+// then to the device.
 hfq_status write_tables(hfq_cache *c, int l, int b, cudaStream_t s)
 {
-    uint64_t *p = c->stage_ptr + (size_t)b * c->E;
-    uint8_t *q = c->stage_loc + (size_t)b * c->E;
+    uint64_t *p = c->stage_ptr + ((size_t)l * 2 + b) * c->E;
+    uint8_t *q = c->stage_loc + ((size_t)l * 2 + b) * c->E;
     for (int e = 0; e < c->E; ++e) {
         p[e] = table_entry(c, l, e);
         q[e] = loc_entry(c, l, e);
@@ -112,16 +115,24 @@ hfq_status hfq_cache_create(int L, int E, size_t expert_bytes, int slots, const 
     c->nobs.assign(L, 0);
     if (table_dev) {
         void *p = nullptr, *q = nullptr;
-        cudaError_t err = cudaHostAlloc(&p, (size_t)2 * E * 8, cudaHostAllocDefault);
-        if (err == cudaSuccess) err = cudaHostAlloc(&q, (size_t)2 * E, cudaHostAllocDefault);
+        cudaError_t err = cudaHostAlloc(&p, (size_t)L * 2 * E * 8, cudaHostAllocDefault);
+        if (err == cudaSuccess) err = cudaHostAlloc(&q, (size_t)L * 2 * E, cudaHostAllocDefault);
         if (err != cudaSuccess) {
             if (p) cudaFreeHost(p);
             delete c;
             return fail(HFQ_ERR_ALLOC, "hfq_cache_create: pinned staging of %zu bytes: %s",
-                        (size_t)2 * E * 9, cudaGetErrorString(err));
+                        (size_t)L * 2 * E * 9, cudaGetErrorString(err));
         }
         c->stage_ptr = static_cast<uint64_t *>(p);
         c->stage_loc = static_cast<uint8_t *>(q);
+        c->staged.assign(L, nullptr);
+        c->staged_live.assign(L, 0);
+        for (int l = 0; l < L && err == cudaSuccess; ++l)
+            err = cudaEventCreateWithFlags(&c->staged[l], cudaEventDisableTiming);
+        if (err != cudaSuccess) {
+            hfq_cache_destroy(c);
+            return fail(HFQ_ERR_CUDA, "hfq_cache_create: events: %s", cudaGetErrorString(err));
+        }
         // nothing cached yet: every table names the experts' homes
         cudaStream_t s = (cudaStream_t)stream;
         for (int l = 0; l < L; ++l) {
@@ -146,11 +157,13 @@ hfq_status hfq_cache_observe(hfq_cache *c, int layer, const int32_t *ids, int n,
         if (ids[i] < 0 || ids[i] >= c->E)
             return fail(HFQ_ERR_ARG, "hfq_cache_observe: expert id %d outside [0, %d)", ids[i], c->E);
     cudaStream_t s = (cudaStream_t)stream;
-    // nothing this cache enqueued earlier may still be pending: the staging
-    // buffers and the bookkeeping are rewritten below
-    if (c->table_dev) {
-        const cudaError_t err = cudaStreamSynchronize(s);
+    // the layer's staging buffers are rewritten below: the copies that read
+    // them in the layer's previous call must have run (nothing else on the
+    // stream is waited for)
+    if (c->table_dev && c->staged_live[layer]) {
+        const cudaError_t err = cudaEventSynchronize(c->staged[layer]);
         if (err != cudaSuccess) return fail(HFQ_ERR_CUDA, "hfq_cache_observe: %s", cudaGetErrorString(err));
+        c->staged_live[layer] = 0;
     }
     const int E = c->E;
     const size_t base = (size_t)layer * E;
@@ -211,6 +224,7 @@ hfq_status hfq_cache_observe(hfq_cache *c, int layer, const int32_t *ids, int n,
         return ok();
     }
     hfq_status st = HFQ_OK;
+    if (!any_evict && admits.empty()) return ok();
     // 1. evicted experts back home (the admitted ones still read from home)
     if (any_evict && (st = write_tables(c, layer, 0, s)) != HFQ_OK) return st;
     // 2. the admitted experts' bytes into their slots (copy engine)
@@ -224,6 +238,9 @@ hfq_status hfq_cache_observe(hfq_cache *c, int layer, const int32_t *ids, int n,
     for (auto &a : admits) c->slot_of[base + a.first] = a.second;
     c->admitted += admits.size();
     if (!admits.empty() && (st = write_tables(c, layer, 1, s)) != HFQ_OK) return st;
+    const cudaError_t err = cudaEventRecord(c->staged[layer], s);
+    if (err != cudaSuccess) return fail(HFQ_ERR_CUDA, "hfq_cache_observe: event: %s", cudaGetErrorString(err));
+    c->staged_live[layer] = 1;
     return ok();
 }
 
@@ -249,6 +266,12 @@ hfq_status hfq_cache_stats(const hfq_cache *c, uint64_t *hits, uint64_t *misses,
 hfq_status hfq_cache_destroy(hfq_cache *c)
 {
     if (!c) return fail(HFQ_ERR_ARG, "hfq_cache_destroy: no cache");
+    // pending copies still read the staging buffers
+    for (size_t l = 0; l < c->staged.size(); ++l)
+        if (c->staged[l]) {
+            if (c->staged_live[l]) cudaEventSynchronize(c->staged[l]);
+            cudaEventDestroy(c->staged[l]);
+        }
     if (c->stage_ptr) cudaFreeHost(c->stage_ptr);
     if (c->stage_loc) cudaFreeHost(c->stage_loc);
     delete c;

@@ -392,8 +392,9 @@ hfq_status hfq_placement_pointers(int L, int E, size_t expert_bytes, const uint8
  * its pinned host address when it lives in host memory (copy source; 0 for
  * experts resident in HBM, which are never cached), and 1 for host experts.
  * table_dev = NULL keeps the bookkeeping only (no device work; policy tests).
- * The library allocates a small host object and a pinned staging buffer of
- * 18 E bytes; hfq_cache_destroy frees them.
+ * The library allocates a small host object, a pinned staging buffer of
+ * 18 L E bytes and L events; hfq_cache_destroy frees them (after the copies
+ * that read the staging have run).
  *
  * hfq_cache_observe: the n expert ids (host array, [0, E)) one step selected
  * in `layer`.  Each distinct selected expert counts as a hit when the kernels
@@ -404,12 +405,16 @@ hfq_status hfq_placement_pointers(int L, int E, size_t expert_bytes, const uint8
  * slot, or in place of the least frequent cached expert not selected in this
  * call when the newcomer is more frequent.  max_admit = -1 admits every
  * missed expert whatever the frequencies (copy-engine staging before use, as
- * long as the slots hold them).  The call first synchronises `stream` (no
- * earlier write of this cache is pending), then enqueues on it: the layer's
- * tables with evicted experts back home, the copies of the admitted experts
- * from pinned host memory into their slots (cudaMemcpyAsync: the copy engine),
- * then the tables naming the admitted experts' slots.  Kernels launched later
- * on `stream` read the new tables; none may run on another stream meanwhile.
+ * long as the slots hold them).  The call waits only for the copies of its
+ * layer's previous call (they read the layer's staging buffers), not for the
+ * rest of `stream`; then it enqueues on `stream`: the layer's tables with
+ * evicted experts back home, the copies of the admitted experts from pinned
+ * host memory into their slots (cudaMemcpyAsync: the copy engine), then the
+ * tables naming the admitted experts' slots.  Kernels enqueued on `stream`
+ * before the call may still run and read the old tables and slot contents
+ * (so a step's routing can be observed while the next step runs); kernels
+ * enqueued after it read the new ones.  None may run on another stream
+ * meanwhile.
  * [CACHE] Strata report, "model and engine": a VRAM cache of hot experts in
  * front of the pinned host arena, refilled from it.
  */
