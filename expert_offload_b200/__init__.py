@@ -77,6 +77,7 @@ _SIGS = {
     "hfq_cache_create": (_i, [_i, _i, _sz, _i, _vp, _vp, _vp, _vp, _sz, _vp, _vp, _vp,
                               ctypes.POINTER(_vp)]),
     "hfq_cache_observe": (_i, [_vp, _i, _vp, _i, _i, _vp]),
+    "hfq_cache_flush": (_i, [_vp, _vp]),
     "hfq_cache_slot_of": (_i, [_vp, _i, _i, ctypes.POINTER(_i)]),
     "hfq_cache_stats": (_i, [_vp, ctypes.POINTER(_u64), ctypes.POINTER(_u64), ctypes.POINTER(_u64),
                              ctypes.POINTER(_u64)]),
@@ -345,6 +346,10 @@ class ExpertCache:
         a = np.ascontiguousarray(ids, np.int32).ravel()
         _check(lib().hfq_cache_observe(self.handle, layer, a.ctypes.data, a.size, max_admit,
                                        _stream(stream)))
+
+    def flush(self, stream=None) -> None:
+        """Names the slots of the refills still in flight."""
+        _check(lib().hfq_cache_flush(self.handle, _stream(stream)))
 
     def slot_of(self, layer: int, expert: int) -> int:
         s = ctypes.c_int()

@@ -37,6 +37,13 @@ struct hfq_cache {
     uint8_t *stage_loc = nullptr;
     std::vector<cudaEvent_t> staged;       // [L]
     std::vector<char> staged_live;         // [L]: the event was recorded
+    // refills (max_admit >= 0 with device tables) copy on their own stream and
+    // name their slots in the layer's next call: [L] admissions in flight, the
+    // events after the layer's evicting table write and after its copies
+    cudaStream_t copy_stream = nullptr;
+    std::vector<std::vector<std::pair<int, int>>> pending;
+    std::vector<cudaEvent_t> evicted_ev, copied_ev;
+    std::vector<int> pending_slot;         // [L][E]: slot of an admission in flight, or -1
     uint64_t hits = 0, misses = 0, admitted = 0, evicted = 0;
 };
 
@@ -73,6 +80,24 @@ hfq_status write_tables(hfq_cache *c, int l, int b, cudaStream_t s)
         err = cudaMemcpyAsync(c->loc_dev + (size_t)l * c->E, q, (size_t)c->E, cudaMemcpyHostToDevice, s);
     if (err != cudaSuccess) return hfq::fail(HFQ_ERR_CUDA, "cache table write: %s", cudaGetErrorString(err));
     return HFQ_OK;
+}
+
+// The layer's admissions in flight name their slots: the tables are written
+// behind their copies (the compute stream waits for the copy stream).
+hfq_status commit_pending(hfq_cache *c, int l, cudaStream_t s)
+{
+    auto &pend = c->pending[l];
+    if (pend.empty()) return HFQ_OK;
+    cudaError_t err = cudaStreamWaitEvent(s, c->copied_ev[l], 0);
+    if (err != cudaSuccess) return hfq::fail(HFQ_ERR_CUDA, "cache commit: %s", cudaGetErrorString(err));
+    const size_t base = (size_t)l * c->E;
+    for (auto &a : pend) {
+        c->slot_of[base + a.first] = a.second;
+        c->pending_slot[base + a.first] = -1;
+    }
+    c->admitted += pend.size();
+    pend.clear();
+    return write_tables(c, l, 1, s);
 }
 
 }  // namespace
@@ -127,8 +152,16 @@ hfq_status hfq_cache_create(int L, int E, size_t expert_bytes, int slots, const 
         c->stage_loc = static_cast<uint8_t *>(q);
         c->staged.assign(L, nullptr);
         c->staged_live.assign(L, 0);
-        for (int l = 0; l < L && err == cudaSuccess; ++l)
+        c->evicted_ev.assign(L, nullptr);
+        c->copied_ev.assign(L, nullptr);
+        c->pending.assign(L, {});
+        c->pending_slot.assign(n, -1);
+        for (int l = 0; l < L && err == cudaSuccess; ++l) {
             err = cudaEventCreateWithFlags(&c->staged[l], cudaEventDisableTiming);
+            if (err == cudaSuccess) err = cudaEventCreateWithFlags(&c->evicted_ev[l], cudaEventDisableTiming);
+            if (err == cudaSuccess) err = cudaEventCreateWithFlags(&c->copied_ev[l], cudaEventDisableTiming);
+        }
+        if (err == cudaSuccess) err = cudaStreamCreateWithFlags(&c->copy_stream, cudaStreamNonBlocking);
         if (err != cudaSuccess) {
             hfq_cache_destroy(c);
             return fail(HFQ_ERR_CUDA, "hfq_cache_create: events: %s", cudaGetErrorString(err));
@@ -167,6 +200,13 @@ hfq_status hfq_cache_observe(hfq_cache *c, int layer, const int32_t *ids, int n,
     }
     const int E = c->E;
     const size_t base = (size_t)layer * E;
+    hfq_status st = HFQ_OK;
+    // the previous call's refills name their slots from the next kernel on
+    bool wrote = false;
+    if (c->table_dev && !c->pending[layer].empty()) {
+        if ((st = commit_pending(c, layer, s)) != HFQ_OK) return st;
+        wrote = true;
+    }
     std::vector<int> cand;                 // missed host experts, once each
     std::vector<char> selected(E, 0);
     for (int i = 0; i < n; ++i) {
@@ -176,6 +216,8 @@ hfq_status hfq_cache_observe(hfq_cache *c, int layer, const int32_t *ids, int n,
         selected[e] = 1;
         if (!c->home_loc[base + e] || c->slot_of[base + e] >= 0) {
             ++c->hits;
+        } else if (c->table_dev && c->pending_slot[base + e] >= 0) {
+            ++c->misses;                               // its copy is in flight
         } else {
             ++c->misses;
             cand.push_back(e);
@@ -202,7 +244,7 @@ hfq_status hfq_cache_observe(hfq_cache *c, int layer, const int32_t *ids, int n,
             int victim = -1;
             for (int q = 0; q < c->slots; ++q) {
                 const int v = owner[q];
-                if (v < 0 || selected[v]) continue;
+                if (v < 0 || selected[v] || (c->table_dev && c->pending_slot[base + v] >= 0)) continue;
                 if (victim < 0 || c->freq[base + v] < c->freq[base + owner[victim]] ||
                     (c->freq[base + v] == c->freq[base + owner[victim]] && v < owner[victim]))
                     victim = q;
@@ -223,10 +265,37 @@ hfq_status hfq_cache_observe(hfq_cache *c, int layer, const int32_t *ids, int n,
         c->admitted += admits.size();
         return ok();
     }
-    hfq_status st = HFQ_OK;
-    if (!any_evict && admits.empty()) return ok();
+    auto record_staged = [&]() -> hfq_status {
+        const cudaError_t err = cudaEventRecord(c->staged[layer], s);
+        if (err != cudaSuccess) return fail(HFQ_ERR_CUDA, "hfq_cache_observe: event: %s", cudaGetErrorString(err));
+        c->staged_live[layer] = 1;
+        return HFQ_OK;
+    };
+    if (!any_evict && admits.empty()) {
+        if (wrote && (st = record_staged()) != HFQ_OK) return st;
+        return ok();
+    }
     // 1. evicted experts back home (the admitted ones still read from home)
     if (any_evict && (st = write_tables(c, layer, 0, s)) != HFQ_OK) return st;
+    if (max_admit >= 0) {
+        // refill: the copies run on the cache's copy stream once the kernels
+        // enqueued so far (which may read the victims' slots) are done; the
+        // slots are named in the layer's next call
+        cudaError_t err = cudaEventRecord(c->evicted_ev[layer], s);
+        if (err == cudaSuccess) err = cudaStreamWaitEvent(c->copy_stream, c->evicted_ev[layer], 0);
+        for (size_t i = 0; i < admits.size() && err == cudaSuccess; ++i) {
+            const auto &a = admits[i];
+            void *dst = c->slot_mem + ((size_t)layer * c->slots + a.second) * c->eb;
+            err = cudaMemcpyAsync(dst, reinterpret_cast<const void *>(c->host_src[base + a.first]), c->eb,
+                                  cudaMemcpyHostToDevice, c->copy_stream);
+            c->pending_slot[base + a.first] = a.second;
+        }
+        if (err == cudaSuccess) err = cudaEventRecord(c->copied_ev[layer], c->copy_stream);
+        if (err != cudaSuccess) return fail(HFQ_ERR_CUDA, "hfq_cache_observe: refill: %s", cudaGetErrorString(err));
+        c->pending[layer] = admits;
+        if ((st = record_staged()) != HFQ_OK) return st;
+        return ok();
+    }
     // 2. the admitted experts' bytes into their slots (copy engine)
     for (auto &a : admits) {
         void *dst = c->slot_mem + ((size_t)layer * c->slots + a.second) * c->eb;
@@ -238,9 +307,28 @@ hfq_status hfq_cache_observe(hfq_cache *c, int layer, const int32_t *ids, int n,
     for (auto &a : admits) c->slot_of[base + a.first] = a.second;
     c->admitted += admits.size();
     if (!admits.empty() && (st = write_tables(c, layer, 1, s)) != HFQ_OK) return st;
-    const cudaError_t err = cudaEventRecord(c->staged[layer], s);
-    if (err != cudaSuccess) return fail(HFQ_ERR_CUDA, "hfq_cache_observe: event: %s", cudaGetErrorString(err));
-    c->staged_live[layer] = 1;
+    if ((st = record_staged()) != HFQ_OK) return st;
+    return ok();
+}
+
+hfq_status hfq_cache_flush(hfq_cache *c, void *stream)
+{
+    if (!c) return fail(HFQ_ERR_ARG, "hfq_cache_flush: no cache");
+    if (!c->table_dev) return ok();
+    cudaStream_t s = (cudaStream_t)stream;
+    for (int l = 0; l < c->L; ++l) {
+        if (c->pending[l].empty()) continue;
+        if (c->staged_live[l]) {
+            const cudaError_t err = cudaEventSynchronize(c->staged[l]);
+            if (err != cudaSuccess) return fail(HFQ_ERR_CUDA, "hfq_cache_flush: %s", cudaGetErrorString(err));
+            c->staged_live[l] = 0;
+        }
+        hfq_status st = commit_pending(c, l, s);
+        if (st != HFQ_OK) return st;
+        const cudaError_t err = cudaEventRecord(c->staged[l], s);
+        if (err != cudaSuccess) return fail(HFQ_ERR_CUDA, "hfq_cache_flush: event: %s", cudaGetErrorString(err));
+        c->staged_live[l] = 1;
+    }
     return ok();
 }
 
@@ -266,12 +354,19 @@ hfq_status hfq_cache_stats(const hfq_cache *c, uint64_t *hits, uint64_t *misses,
 hfq_status hfq_cache_destroy(hfq_cache *c)
 {
     if (!c) return fail(HFQ_ERR_ARG, "hfq_cache_destroy: no cache");
-    // pending copies still read the staging buffers
-    for (size_t l = 0; l < c->staged.size(); ++l)
+    // pending copies still read the staging buffers or write the slots
+    if (c->copy_stream) {
+        cudaStreamSynchronize(c->copy_stream);
+        cudaStreamDestroy(c->copy_stream);
+    }
+    for (size_t l = 0; l < c->staged.size(); ++l) {
         if (c->staged[l]) {
             if (c->staged_live[l]) cudaEventSynchronize(c->staged[l]);
             cudaEventDestroy(c->staged[l]);
         }
+        if (c->evicted_ev[l]) cudaEventDestroy(c->evicted_ev[l]);
+        if (c->copied_ev[l]) cudaEventDestroy(c->copied_ev[l]);
+    }
     if (c->stage_ptr) cudaFreeHost(c->stage_ptr);
     if (c->stage_loc) cudaFreeHost(c->stage_loc);
     delete c;

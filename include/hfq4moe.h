@@ -393,8 +393,8 @@ hfq_status hfq_placement_pointers(int L, int E, size_t expert_bytes, const uint8
  * experts resident in HBM, which are never cached), and 1 for host experts.
  * table_dev = NULL keeps the bookkeeping only (no device work; policy tests).
  * The library allocates a small host object, a pinned staging buffer of
- * 18 L E bytes and L events; hfq_cache_destroy frees them (after the copies
- * that read the staging have run).
+ * 18 L E bytes, 3 L events and one stream for refill copies;
+ * hfq_cache_destroy waits for its copies and frees them.
  *
  * hfq_cache_observe: the n expert ids (host array, [0, E)) one step selected
  * in `layer`.  Each distinct selected expert counts as a hit when the kernels
@@ -405,16 +405,22 @@ hfq_status hfq_placement_pointers(int L, int E, size_t expert_bytes, const uint8
  * slot, or in place of the least frequent cached expert not selected in this
  * call when the newcomer is more frequent.  max_admit = -1 admits every
  * missed expert whatever the frequencies (copy-engine staging before use, as
- * long as the slots hold them).  The call waits only for the copies of its
- * layer's previous call (they read the layer's staging buffers), not for the
- * rest of `stream`; then it enqueues on `stream`: the layer's tables with
- * evicted experts back home, the copies of the admitted experts from pinned
- * host memory into their slots (cudaMemcpyAsync: the copy engine), then the
- * tables naming the admitted experts' slots.  Kernels enqueued on `stream`
- * before the call may still run and read the old tables and slot contents
- * (so a step's routing can be observed while the next step runs); kernels
- * enqueued after it read the new ones.  None may run on another stream
- * meanwhile.
+ * long as the slots hold them).  The call waits only for the table copies
+ * of its layer's previous call (they read the layer's staging buffers), not
+ * for the rest of `stream`.  Then it enqueues on `stream` the layer's tables
+ * with evicted experts back home.  With max_admit = -1 it then enqueues on
+ * `stream` the copies of the admitted experts from pinned host memory into
+ * their slots (cudaMemcpyAsync: the copy engine) and the tables naming those
+ * slots, so the next kernel reads them from HBM.  With max_admit >= 0
+ * (refill) the copies run on the cache's own stream, behind every kernel
+ * enqueued on `stream` so far (they may still read the victims' slots), and
+ * overlap the kernels enqueued next.  Their slots are named at the start of
+ * the layer's next call, or by hfq_cache_flush, behind those copies; until
+ * then the kernels read those experts from their homes and
+ * hfq_cache_slot_of reports -1 for them.  Kernels enqueued on `stream`
+ * before a call may still run and read the old tables and slot contents, so
+ * a step's routing can be observed while the next step runs.  No kernel that
+ * reads these tables may run on another stream.
  * [CACHE] Strata report, "model and engine": a VRAM cache of hot experts in
  * front of the pinned host arena, refilled from it.
  */
@@ -425,7 +431,10 @@ hfq_status hfq_cache_create(int L, int E, size_t expert_bytes, int slots, const 
                             hfq_cache **out);
 hfq_status hfq_cache_observe(hfq_cache *cache, int layer, const int32_t *ids, int n, int max_admit,
                              void *stream);
-/* Slot of an expert (-1: not cached). */
+/* Names the slots of every layer's refills in flight (see hfq_cache_observe),
+ * enqueued on `stream` behind their copies. */
+hfq_status hfq_cache_flush(hfq_cache *cache, void *stream);
+/* Slot of an expert (-1: not cached, or its refill not yet named). */
 hfq_status hfq_cache_slot_of(const hfq_cache *cache, int layer, int expert, int *slot);
 /* Counters since creation (any pointer may be NULL). */
 hfq_status hfq_cache_stats(const hfq_cache *cache, uint64_t *hits, uint64_t *misses,

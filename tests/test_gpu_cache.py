@@ -1,7 +1,8 @@
 """The expert cache on the GPU: the decode stack over cache-managed pointer
 tables gives the same bits as over the plain host-mapped tables, while the
-copy engine moves experts into HBM slots and the tables switch between a
-slot and the expert's host alias (Strata report, "model and engine": a VRAM
+copy engine moves experts into HBM slots (refills on the cache's own stream,
+named one call later) and the tables switch between a slot and the expert's
+host alias (Strata report, "model and engine": a VRAM
 cache of hot experts in front of the pinned host arena; hipfire offload
 explainer, "PCIe pass-through": the zero-copy reads it competes with)."""
 import numpy as np
@@ -89,6 +90,14 @@ def test_cache_managed_tables_give_the_same_bits(eo, host_model, max_admit):
             if max_admit >= 0:
                 for l in range(L):
                     cache.observe(l, idx_c[l].ravel(), max_admit)
+        if max_admit >= 0:
+            # refills in flight are named by the flush; the tables then still
+            # give the same bits
+            cache.flush()
+            named = [(l, e) for l in range(L) for e in range(E) if cache.slot_of(l, e) >= 0]
+            assert named
+            y_c, _ = _stack(eo, layers, d_logits, d_x0, k, H, I, E)
+            np.testing.assert_array_equal(y_c.view(np.uint32), y_z.view(np.uint32))
         st = cache.stats()
         assert st["admitted"] > 0 and st["hits"] > 0
         # and the values themselves against the oracle, last token
