@@ -276,8 +276,8 @@ hfq_status hfq4_moe_decode_stack_routed(const hfq4_layer *layers, int n_layers, 
  *   Limits: 1 <= T <= 8, k <= 16, inter <= 1024, hidden <= 2048; anything
  *   larger returns HFQ_ERR_UNSUPPORTED naming the limit.
  *   The first call on a device looks up the array's device address for that
- *   device (with that device current); make that first call before any stream
- *   capture.  Each call clears the array's control words on `stream` before
+ *   device (with that device current).  Each call clears the array's control
+ *   words on `stream` before
  *   launching, the status word among them.  All calls share the one array, so
  *   calls that overlap on the GPU (different streams without ordering) race;
  *   order them on one stream.  Calls may change k, T and the layer's shape

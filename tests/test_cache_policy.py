@@ -104,3 +104,11 @@ def test_bad_ids_are_refused():
         c.observe(0, [3, 9], 1)
     assert e.value.status == -1
     c.close()
+
+
+def test_flush_without_device_tables_is_a_no_op():
+    c = _cache(1, 4, 2, [1] * 4)
+    c.observe(0, [0, 1], 2)
+    c.flush()
+    assert c.slot_of(0, 0) >= 0 and c.slot_of(0, 1) >= 0
+    c.close()
