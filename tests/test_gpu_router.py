@@ -97,13 +97,15 @@ def test_router_logits_rejects_bad_arguments(eo):
     assert e.value.status == -2            # HFQ_ERR_ALIGN
 
 
-@pytest.fixture(scope="module")
-def stack_model(eo):
-    """The first four layers of the 40-layer decode model (H 2048, I 512,
-    E 256, top-8), resident in HBM."""
+@pytest.fixture(scope="module", params=[2, 3, 1], ids=["decode_e256", "verify_e512", "tiny_e16"])
+def stack_model(eo, request):
+    """A prefix of a model, resident in HBM: the 40-layer decode model (H 2048,
+    I 512, E 256, top-8; 4 layers), the 48-layer verify model (E 512: up to 4
+    router rows per CTA; 3 layers) and the tiny layer (H 256, I 128, E 16,
+    top-4: most CTAs own no router row)."""
     from expert_offload_b200.model import ExpertStore
-    w = W.WORKLOADS[2]
-    L = 4
+    w = W.WORKLOADS[request.param]
+    L = min({2: 4, 3: 3, 1: 1}[request.param], w.layers)
     store = ExpertStore(torch, L, w.experts, w.hidden, w.inter, device_fill(torch, w))
     caches = [moe.ExpertCache(OraclePackedLayer(w, l), w.hidden, w.inter) for l in range(L)]
     yield w, L, store, caches
@@ -177,7 +179,7 @@ def test_routed_stack(eo, stack_model, T, r_bf16):
     w, L, store, caches = stack_model
     H, I, E, k = w.hidden, w.inter, w.experts, w.top_k
     wr_dev, wr_val = _router(w, L, r_bf16)
-    x0, _ = W.activations(w, 300, T)
+    x0 = synth.to_bf16_bits(W.activations_f32(w, 300, T))       # bf16 residual stream
     x0_val = synth.bf16_bits_to_f32(x0)
     d_x0 = torch.from_numpy(x0.view(np.int16)).cuda()
     d_wr = torch.from_numpy(np.ascontiguousarray(wr_dev.view(np.int16) if r_bf16 else wr_dev)).cuda()
