@@ -72,7 +72,8 @@ struct VArgs {
     int L, T, E, k, H, I;
     int extra_arrivals;       // test hook: grid barriers wait for this many more CTAs
     int NS, stage_bytes;      // ring
-    int xp_off, xres_off, ysh_off, hst_off, sh_off;
+    int xp_off, xres_off, ysh_off, hst_off, tab_off, sh_off;
+    int tab_pref;             // the layers' expert tables are prefetched into shared memory
     unsigned long long *timeline;   // debug: [G][L][32] %globaltimer stamps, or null
 };
 
@@ -165,7 +166,20 @@ __device__ __forceinline__ void build_x_piece(const float (&v)[8], uint32_t *pie
 
 // Warp 0: unique experts of the layer (ascending), their token masks and slot
 // per token, and the pairs in (expert, token) order.
-__device__ void build_pairs(VShared &sh, const VArgs &a, int l)
+// Layer l's expert table (and location table) into shared memory, one
+// cp.async group of warp 0, waited for in build_pairs: the table of the next
+// layer travels while this one's down items compute.
+__device__ __forceinline__ void fetch_tables(const VArgs &a, int l, uint8_t *tab)
+{
+    const int lane = threadIdx.x & 31;
+    const uint8_t *src = reinterpret_cast<const uint8_t *>(a.eptr[l]);
+    for (int i = lane; i < a.E / 2; i += 32) cp_async16(tab + 16 * i, src + 16 * i);
+    if (a.eloc[l])
+        for (int i = lane; i < a.E / 16; i += 32) cp_async16(tab + (size_t)a.E * 8 + 16 * i, a.eloc[l] + 16 * i);
+    cp_async_commit();
+}
+
+__device__ void build_pairs(VShared &sh, const VArgs &a, int l, const uint8_t *tab)
 {
     const int lane = threadIdx.x & 31, T = a.T, k = a.k;
     if (lane < HFQ_MAX_EXPERTS / 32) sh.ebits[lane] = 0u;
@@ -194,11 +208,20 @@ __device__ void build_pairs(VShared &sh, const VArgs &a, int l)
         atomicOr(&sh.umask[u], 1u << t);
     }
     __syncwarp();
-    // expert bases and locations, one round of loads
+    // expert bases and locations: from the prefetched tables, or one round of loads
+    if (a.tab_pref) {
+        cp_async_wait_all();
+        __syncwarp();
+    }
     for (int u = lane; u < U; u += 32) {
         const int e = sh.uexp[u];
-        sh.ubase[u] = static_cast<const uint8_t *>(a.eptr[l][e]);
-        sh.uloc[u] = a.eloc[l] ? a.eloc[l][e] : 0;
+        if (a.tab_pref) {
+            sh.ubase[u] = reinterpret_cast<const uint8_t *const *>(tab)[e];
+            sh.uloc[u] = a.eloc[l] ? tab[(size_t)a.E * 8 + e] : 0;
+        } else {
+            sh.ubase[u] = static_cast<const uint8_t *>(a.eptr[l][e]);
+            sh.uloc[u] = a.eloc[l] ? a.eloc[l][e] : 0;
+        }
     }
     // pairs: lane u (then u + 32) writes expert u's pairs at its prefix offset
     int run = 0;
@@ -255,6 +278,7 @@ __global__ void __launch_bounds__(kThr, 1) verify_kernel(const __grid_constant__
     float *ysh = reinterpret_cast<float *>(smem + a.ysh_off);         // [kCW][T][kMaxDRows]
     float *hst = reinterpret_cast<float *>(smem + a.hst_off);         // [kCW][2][nbI*4][kHStride]
     VShared &sh = *reinterpret_cast<VShared *>(smem + a.sh_off);
+    uint8_t *tab = smem + a.tab_off;                                   // [E] u64 expert table, [E] u8 locations
     const WaitCtx wc{a.ctl, a.timeout_ns, &sh.abort};
 
     if (tid == 0) {
@@ -266,6 +290,7 @@ __global__ void __launch_bounds__(kThr, 1) verify_kernel(const __grid_constant__
         sh.abort = 0;
         fence_mbar_init();
     }
+    if (warp == 0 && a.tab_pref) fetch_tables(a, 0, tab);
     __syncthreads();
 
     int stage_base = 0;                 // ring items of earlier layers (same in every warp)
@@ -336,7 +361,7 @@ __global__ void __launch_bounds__(kThr, 1) verify_kernel(const __grid_constant__
         }
         __syncthreads();
         vstamp(a, l, 1, tid == 0);
-        if (warp == 0) build_pairs(sh, a, l);
+        if (warp == 0) build_pairs(sh, a, l, tab);
         if (__syncthreads_or(sh.abort)) break;
         vstamp(a, l, 2, tid == 0);
         const int U = sh.U, P = sh.P;
@@ -608,6 +633,8 @@ __global__ void __launch_bounds__(kThr, 1) verify_kernel(const __grid_constant__
             }
             cp_async_wait_all();
             if (!ok) sh.abort = 1;
+            // the next layer's tables travel while the other warps finish
+            if (warp == 0 && a.tab_pref && l + 1 < a.L) fetch_tables(a, l + 1, tab);
         }
         stage_base += 2 * U;
         __syncthreads();
@@ -643,7 +670,8 @@ __global__ void __launch_bounds__(kThr, 1) verify_kernel(const __grid_constant__
     }
 
     // no copy may still be writing this CTA's shared memory when it exits:
-    // every stage's last armed phase completes (bounded)
+    // the tables' cp.async group, and every stage's last armed phase (bounded)
+    cp_async_wait_all();
     __syncthreads();
     if (tid < NS) {
         const int seq = sh.armed_seq[tid];
@@ -724,7 +752,8 @@ hfq_status verify_launch(const hfq4_layer *layers, int L, const float *logits, c
     const size_t xres_b = (size_t)T * kMaxDRows * 4;
     const size_t ysh_b = (size_t)kCW * T * kMaxDRows * 4;
     const size_t hst_b = (size_t)kCW * 2 * nbI * 4 * kHStride * 4;
-    fixed = xp_b + xres_b + ysh_b + hst_b + up128(sizeof(VShared));
+    const size_t tab_b = up128((size_t)E * 9);
+    fixed = xp_b + xres_b + ysh_b + hst_b + tab_b + up128(sizeof(VShared));
 
     static int dyn_limit = 0;
     if (!dyn_limit) {
@@ -749,6 +778,12 @@ hfq_status verify_launch(const hfq4_layer *layers, int L, const float *logits, c
     a.xres_off = (int)off; off += xres_b;
     a.ysh_off = (int)off; off += ysh_b;
     a.hst_off = (int)off; off += hst_b;
+    a.tab_off = (int)up128(off); off = (size_t)a.tab_off + tab_b;
+    // prefetched tables: 16-byte copies of whole tables
+    a.tab_pref = E % 16 == 0;
+    for (int l = 0; l < L; ++l)
+        if (!aligned16(layers[l].expert_ptr) || (layers[l].expert_loc && !aligned16(layers[l].expert_loc)))
+            a.tab_pref = 0;
     a.sh_off = (int)up128(off);
     const size_t smem = (size_t)a.sh_off + sizeof(VShared);
     if (smem > (size_t)dyn_limit) return HFQ_ERR_UNSUPPORTED;
