@@ -509,9 +509,9 @@ def run_headline(args, rank, world, local_rank, dist):
 
 # DRAM traffic of one decode1_kernel launch on the headline workload, or None
 # while no capture of the current kernel exists (see profiles/).
-TRAFFIC_DECODE_L40 = 4 * (133871360 + 2799616)
-TRAFFIC_SOURCE = ("ncu dram__bytes_read.sum + dram__bytes_write.sum of one decode1_kernel launch "
-                  "over the first 10 layers (133,871,360 + 2,799,616 B), x 4")
+TRAFFIC_DECODE_L40 = 4 * (133841920 + 3118336)
+TRAFFIC_SOURCE = ("ncu dram__bytes_read.sum + dram__bytes_write.sum of one decode1_kernel<0, 1> launch "
+                  "over the first 10 layers (133,841,920 + 3,118,336 B), x 4")
 
 
 # --------------------------------------------------------- the other configs
