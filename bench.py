@@ -509,9 +509,9 @@ def run_headline(args, rank, world, local_rank, dist):
 
 # DRAM traffic of one decode1_kernel launch on the headline workload, or None
 # while no capture of the current kernel exists (see profiles/).
-TRAFFIC_DECODE_L40 = 4 * (133841920 + 3118336)
-TRAFFIC_SOURCE = ("ncu dram__bytes_read.sum + dram__bytes_write.sum of one decode1_kernel<0, 1> launch "
-                  "over the first 10 layers (133,841,920 + 3,118,336 B), x 4")
+TRAFFIC_DECODE_L40 = 4 * (133848064 + 3205632)
+TRAFFIC_SOURCE = ("ncu dram__bytes_read.sum + dram__bytes_write.sum of one decode1_kernel<0, 1, 0> launch "
+                  "over the first 10 layers (133,848,064 + 3,205,632 B), x 4")
 
 
 # --------------------------------------------------------- the other configs

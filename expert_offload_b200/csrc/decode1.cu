@@ -164,9 +164,10 @@ __device__ __forceinline__ Span span_of(size_t off, size_t len)
     return s;
 }
 
+template <bool kOn>
 __device__ __forceinline__ void stamp(const D1Args &a, int l, int s)
 {
-    if (a.timeline && threadIdx.x == 0 && l < a.L) {
+    if (kOn && a.timeline && threadIdx.x == 0 && l < a.L) {
         const int slot = blockIdx.x == 0 ? 0 : (blockIdx.x == gridDim.x / 2 ? 1 : -1);
         if (slot >= 0) a.timeline[((size_t)slot * a.L + l) * kStamps + s] = globaltimer_ns();
     }
@@ -174,9 +175,10 @@ __device__ __forceinline__ void stamp(const D1Args &a, int l, int s)
 
 // Debug timeline, thread `who` of CTAs 0 and G/2: %globaltimer once `dep`
 // (a value the stamp waits for) is available.
+template <bool kOn>
 __device__ __forceinline__ void stamp_dep(const D1Args &a, int l, int s, bool who, float dep)
 {
-    if (a.timeline && who && l < a.L) {
+    if (kOn && a.timeline && who && l < a.L) {
         const int slot = blockIdx.x == 0 ? 0 : (blockIdx.x == gridDim.x / 2 ? 1 : -1);
         if (slot >= 0) {
             uint64_t t;
@@ -218,9 +220,11 @@ __device__ __forceinline__ void fetch_table(const D1Args &a, int l, uint8_t *pta
 }
 
 // kRouter: the launch computes the logits (a.router set); kSmallK: k <= kW
-// routing.  One instantiation per combination keeps the code a launch runs
-// small (fewer instruction-cache misses: about 2 % of a step).
-template <bool kRouter, bool kSmallK>
+// routing; kFull: host-mapped experts or the debug timeline are possible.
+// One instantiation per combination keeps the code a launch runs small
+// (instruction-cache misses were the largest stall reason): the router and
+// rank routing out cut a step by 2 %, the host paths and stamps out by 4 %.
+template <bool kRouter, bool kSmallK, bool kFull>
 __global__ void __launch_bounds__(kThr, 1) decode1_kernel(const __grid_constant__ D1Args a)
 {
     extern __shared__ __align__(1024) uint8_t smem[];
@@ -298,7 +302,7 @@ __global__ void __launch_bounds__(kThr, 1) decode1_kernel(const __grid_constant_
     const int n_layers = __syncthreads_or(sh.abort) ? 0 : a.L;
 
     for (int l = 0; l < n_layers; ++l) {
-        stamp(a, l, 0);
+        stamp<kFull>(a, l, 0);
         const uint32_t par = l & 1;          // parity of this layer's slot-barrier phases
         // ---------------------------------------------- 1a. layer input -> xs
         if (l == 0) {
@@ -356,7 +360,7 @@ __global__ void __launch_bounds__(kThr, 1) decode1_kernel(const __grid_constant_
             }
         }
         if (__syncthreads_or(sh.abort)) break;
-        stamp(a, l, 4);
+        stamp<kFull>(a, l, 4);
         // ---------------------------------------------- 1a'. router (optional)
         // logits = Wr_l x_l for experts [r_lo, r_hi) from this CTA's rows in
         // rsm, in the summation order of moe_router_logits (same bits):
@@ -429,7 +433,7 @@ __global__ void __launch_bounds__(kThr, 1) decode1_kernel(const __grid_constant_
                 }
             }
             if (__syncthreads_or(sh.abort)) break;
-            stamp(a, l, 31);
+            stamp<kFull>(a, l, 31);
             // rsm is free again: the next layer's rows travel during this layer
             if (tid == 0 && l + 1 < n_layers) {
                 fence_proxy_async_smem();
@@ -453,11 +457,11 @@ __global__ void __launch_bounds__(kThr, 1) decode1_kernel(const __grid_constant_
             // ------------------------------------------ 1c. issue copies
             cp_async_wait_all();
             __syncwarp();
-            stamp_dep(a, l, 29, lane == 0, 0.f);
+            stamp_dep<kFull>(a, l, 29, lane == 0, 0.f);
             int e = re;
             float w = rw;
             if (a.idx_in && lane < k) { e = a.idx_in[lane]; w = a.wts_in[lane]; }
-            stamp_dep(a, l, 2, lane == 0, w);
+            stamp_dep<kFull>(a, l, 2, lane == 0, w);
             bool bad = lane < k && (unsigned)e >= (unsigned)E;
             const uint8_t *base = nullptr;
             int loc = 0;
@@ -470,7 +474,7 @@ __global__ void __launch_bounds__(kThr, 1) decode1_kernel(const __grid_constant_
                 __syncwarp();
             }
             if (lane < k && !bad) {
-                loc = a.eloc[l] ? ltab[(size_t)par * a.ltab_stride + e] : 0;
+                loc = kFull && a.eloc[l] ? ltab[(size_t)par * a.ltab_stride + e] : 0;
                 sh.base[lane] = base;
                 sh.w[lane] = w;
                 if (a.idx_all && c == 0) {
@@ -480,7 +484,7 @@ __global__ void __launch_bounds__(kThr, 1) decode1_kernel(const __grid_constant_
             }
             const unsigned hm = __ballot_sync(0xffffffffu, lane < k && loc != 0);
             __syncwarp();
-            stamp_dep(a, l, 25, lane == 0, 0.f);
+            stamp_dep<kFull>(a, l, 25, lane == 0, 0.f);
             if (!sh.abort) {
                 // the slots were last read by the generic proxy (previous layer)
                 fence_proxy_async_smem();
@@ -495,7 +499,7 @@ __global__ void __launch_bounds__(kThr, 1) decode1_kernel(const __grid_constant_
                     }
                 }
                 __syncwarp();
-                stamp_dep(a, l, 26, lane == 0, 0.f);
+                stamp_dep<kFull>(a, l, 26, lane == 0, 0.f);
                 if (lane < k && !loc) {
                     // expert bytes are read once per step: evict them first from L2
                     const uint64_t pol = l2_evict_first_policy();
@@ -505,12 +509,12 @@ __global__ void __launch_bounds__(kThr, 1) decode1_kernel(const __grid_constant_
                 }
                 if (lane == 0) { sh.armed = l + 1; sh.hostmask = hm; }
                 __syncwarp();
-                stamp_dep(a, l, 27, lane == 0, 0.f);
+                stamp_dep<kFull>(a, l, 27, lane == 0, 0.f);
             }
             // next layer's table, after the copies: the proxy fence above must
             // not wait for it
             if (l + 1 < a.L) fetch_table(a, l + 1, ptab, ltab);
-            stamp_dep(a, l, 3, lane == 0, 0.f);
+            stamp_dep<kFull>(a, l, 3, lane == 0, 0.f);
         }
 
         // ---------------------------------------------- 2. gate/up rows
@@ -543,11 +547,11 @@ __global__ void __launch_bounds__(kThr, 1) decode1_kernel(const __grid_constant_
         // warps 1..7 prepared their activations while warp 0 routed; the
         // routing's slot table is complete after this
         if (__syncthreads_or(sh.abort)) break;
-        stamp(a, l, 1);
+        stamp<kFull>(a, l, 1);
         bool ok = true;
         for (int j = warp; j < k && ok; j += kW) {
             uint8_t *slot = slots + (size_t)j * a.slot_bytes;
-            if (sh.hostmask >> j & 1u) {
+            if (kFull && (sh.hostmask >> j & 1u)) {
                 warp_copy_host(slot, sh.base[j] + sg.src, sg.len);
                 warp_copy_host(slot + a.up_off, sh.base[j] + su.src, su.len);
             } else if (!wait_mbar_phase(wc, &sh.gu_bar[j], par)) {
@@ -560,7 +564,7 @@ __global__ void __launch_bounds__(kThr, 1) decode1_kernel(const __grid_constant_
                 bulk_g2s_hint(slot + a.down_off, sh.base[j] + sd.src, (uint32_t)sd.len, &sh.d_bar[j],
                               l2_evict_first_policy());
             }
-            stamp_dep(a, l, 5 + j, lane == 0 && (warp == 0 || warp == 7), 0.f);
+            stamp_dep<kFull>(a, l, 5 + j, lane == 0 && (warp == 0 || warp == 7), 0.f);
             const uint8_t *g0 = slot + sg.delta, *u0 = slot + a.up_off + su.delta;
             for (int r0 = 0; r0 < n_gu; r0 += kGuRows) {
                 constexpr int kD = 2 * kGuRows;      // the group's dots: gate rows, then up rows
@@ -602,14 +606,14 @@ __global__ void __launch_bounds__(kThr, 1) decode1_kernel(const __grid_constant_
             }
         }
         if (__syncthreads_or(!ok || sh.abort)) break;
-        stamp(a, l, 16);
+        stamp<kFull>(a, l, 16);
 
         // ---------------------------------------------- 3. h exchange, down rows
         // down rows of host slots travel while other CTAs finish their h rows
         for (int j = warp; j < k; j += kW)
-            if (sh.hostmask >> j & 1u)
+            if (kFull && (sh.hostmask >> j & 1u))
                 warp_copy_host(slots + (size_t)j * a.slot_bytes + a.down_off, sh.base[j] + sd.src, sd.len);
-        stamp(a, l, 17);
+        stamp<kFull>(a, l, 17);
 
         // this warp's weighted row sums, ysh[warp][ri], summed over its slots.
         // Lane: piece pc (64 values of h, one quarter of a block) of row rs of
@@ -692,12 +696,12 @@ __global__ void __launch_bounds__(kThr, 1) decode1_kernel(const __grid_constant_
                 }
             }
             __syncwarp();                              // the staging row is read; next slot may overwrite
-            stamp_dep(a, l, 21, lane == 0 && warp == 0, hs2.x);
-            if (!(sh.hostmask >> j & 1u) && !wait_mbar_phase(wc, &sh.d_bar[j], par)) {
+            stamp_dep<kFull>(a, l, 21, lane == 0 && warp == 0, hs2.x);
+            if (!(kFull && (sh.hostmask >> j & 1u)) && !wait_mbar_phase(wc, &sh.d_bar[j], par)) {
                 ok = false;
                 break;
             }
-            stamp_dep(a, l, 22, lane == 0 && warp == 0, 0.f);
+            stamp_dep<kFull>(a, l, 22, lane == 0 && warp == 0, 0.f);
             const uint8_t *d0 = slots + (size_t)j * a.slot_bytes + a.down_off + sd.delta +
                                 (pc >> 2) * kBlockBytes;                 // this lane's block of each row
             const float wj = sh.w[j];
@@ -727,9 +731,9 @@ __global__ void __launch_bounds__(kThr, 1) decode1_kernel(const __grid_constant_
                 }
             }
         }
-        stamp_dep(a, l, 23, lane == 0 && warp == 0, ysh[warp * kMaxDRows]);
+        stamp_dep<kFull>(a, l, 23, lane == 0 && warp == 0, ysh[warp * kMaxDRows]);
         if (__syncthreads_or(!ok || sh.abort)) break;
-        stamp(a, l, 19);
+        stamp<kFull>(a, l, 19);
 
         // ---------------------------------------------- 4. combine, residual
         if (tid < n_d) {
@@ -747,7 +751,7 @@ __global__ void __launch_bounds__(kThr, 1) decode1_kernel(const __grid_constant_
                 st_tagged(a.xbuf + (size_t)((l + 1) & 1) * H + r, __uint_as_float(xb), xch_tag(epoch, l + 1));
             }
         }
-        stamp(a, l, 20);
+        stamp<kFull>(a, l, 20);
         // xs and ysh are read by the combine before the next layer rewrites them
         if (l + 1 < a.L && __syncthreads_or(sh.abort)) break;
     }
@@ -872,11 +876,16 @@ hfq_status decode1_launch(const hfq4_layer *layers, int L, const float *logits, 
     const size_t smem = (size_t)a.sh_off + sizeof(D1Shared);
 
     // the instantiation for this launch, and its shared-memory limit (set once)
-    const int variant = (router ? 2 : 0) + (k <= kW ? 1 : 0);
-    const void *const kernels[4] = {(const void *)decode1_kernel<false, false>, (const void *)decode1_kernel<false, true>,
-                                    (const void *)decode1_kernel<true, false>, (const void *)decode1_kernel<true, true>};
+    bool full = a.timeline != nullptr;
+    for (int l = 0; l < L; ++l) full = full || layers[l].expert_loc != nullptr;
+    const int variant = (router ? 4 : 0) + (k <= kW ? 2 : 0) + (full ? 1 : 0);
+    const void *const kernels[8] = {
+        (const void *)decode1_kernel<false, false, false>, (const void *)decode1_kernel<false, false, true>,
+        (const void *)decode1_kernel<false, true, false>,  (const void *)decode1_kernel<false, true, true>,
+        (const void *)decode1_kernel<true, false, false>,  (const void *)decode1_kernel<true, false, true>,
+        (const void *)decode1_kernel<true, true, false>,   (const void *)decode1_kernel<true, true, true>};
     const void *kernel = kernels[variant];
-    static int dyn_limit[4] = {0, 0, 0, 0};
+    static int dyn_limit[8] = {0, 0, 0, 0, 0, 0, 0, 0};
     if (!dyn_limit[variant]) {
         int dev = 0, optin = 0;
         cudaGetDevice(&dev);
