@@ -65,7 +65,7 @@ struct D1Args {
     float *logits_out;        // [L][E] the computed logits (router), or null
     const int32_t *idx_in;    // [k] given routing (single layer), or null
     const float *wts_in;
-    const void *x0;           // [H] bf16 (f32 when x0_f32)
+    const void *x0;           // [H] bf16
     uint16_t *x_out;          // [H] bf16 input of the layer after the last, or null
     uint64_t *xbuf;           // [2][H] {bf16 value, tag} words, ping-pong between layers (L > 1)
     uint64_t *h;              // [2][k][Ip] {f32 value, tag} words, ping-pong between layers
@@ -77,7 +77,6 @@ struct D1Args {
     long long timeout_ns;
     unsigned long long *timeline;   // debug: [2][L][kStamps] %globaltimer stamps, or null
     int L, E, k, H, I;
-    int x0_f32;
     int extra_arrivals;       // test hook: nonzero makes the layer-1 input poll (one layer: the h poll)
                               // expect a tag nobody writes
     // shared-memory layout, bytes; a slot is [gate span][up span][down span]
@@ -220,7 +219,8 @@ __device__ __forceinline__ void fetch_table(const D1Args &a, int l, uint8_t *pta
 }
 
 // kRouter: the launch computes the logits (a.router set); kSmallK: k <= kW
-// routing; kFull: host-mapped experts or the debug timeline are possible.
+// routing; kFull: host-mapped experts, given routing, the debug timeline or
+// the test hook are possible.
 // One instantiation per combination keeps the code a launch runs small
 // (instruction-cache misses were the largest stall reason): the router and
 // rank routing out cut a step by 2 %, the host paths and stamps out by 4 %.
@@ -256,7 +256,9 @@ __global__ void __launch_bounds__(kThr, 1) decode1_kernel(const __grid_constant_
     const bool reset = *(volatile const unsigned *)(a.ctl + kCtlSig) != sig;
     // router: CTA c computes the logits of experts [r_lo, r_hi); their Wr rows
     // are one contiguous span, copied into rsm a layer ahead
-    const bool route_in_kernel = kRouter && !a.idx_in;
+    // given routing (a single layer's forward) only in the full instantiation
+    const int32_t *const idx_in = kFull ? a.idx_in : nullptr;
+    const bool route_in_kernel = kRouter && !idx_in;
     const int r_lo = (int)((long long)c * E / G), r_hi = (int)((long long)(c + 1) * E / G);
     const uint32_t r_len = route_in_kernel ? (uint32_t)((r_hi - r_lo) * H * 2) : 0u;
     auto issue_router = [&](int l) {       // thread 0
@@ -306,28 +308,21 @@ __global__ void __launch_bounds__(kThr, 1) decode1_kernel(const __grid_constant_
         const uint32_t par = l & 1;          // parity of this layer's slot-barrier phases
         // ---------------------------------------------- 1a. layer input -> xs
         if (l == 0) {
-            const bool f32 = a.x0_f32;
-            const int per = f32 ? 4 : 8;                // values per 16-byte load
-            const int nld = H / per;
-            for (int i = tid; i < nld; i += kThr) {
+            // bf16 input, 8 values per 16-byte load
+            for (int i = tid; i < H / 8; i += kThr) {
                 const uint4 v = __ldcg(static_cast<const uint4 *>(a.x0) + i);
-                float2 *dst = reinterpret_cast<float2 *>(xs + xp4(i * per));
-                if (f32) {
-                    dst[0] = make_float2(__uint_as_float(v.x), __uint_as_float(v.y));
-                    dst[1] = make_float2(__uint_as_float(v.z), __uint_as_float(v.w));
-                } else {
-                    const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+                float2 *dst = reinterpret_cast<float2 *>(xs + xp4(i * 8));
+                const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-                    for (int r = 0; r < 4; ++r)
-                        dst[r] = make_float2(__uint_as_float(w4[r] << 16), __uint_as_float(w4[r] & 0xFFFF0000u));
-                }
+                for (int r = 0; r < 4; ++r)
+                    dst[r] = make_float2(__uint_as_float(w4[r] << 16), __uint_as_float(w4[r] & 0xFFFF0000u));
             }
         } else {
             // poll the tagged words of x_l (pairs 2 i, 2 i + 1, i = tid + kThr m)
             // until every one carries layer l's tag: then every CTA has
             // finished layer l - 1 (the test hook expects a tag nobody writes)
             const uint64_t *xw = a.xbuf + (size_t)(l & 1) * H;
-            const uint32_t tag = xch_tag(epoch, l) ^ (a.extra_arrivals && l == 1 ? 1u : 0u);
+            const uint32_t tag = xch_tag(epoch, l) ^ (kFull && a.extra_arrivals && l == 1 ? 1u : 0u);
             unsigned pend = 0;
 #pragma unroll
             for (int m = 0; m < kXLoads; ++m)
@@ -445,7 +440,7 @@ __global__ void __launch_bounds__(kThr, 1) decode1_kernel(const __grid_constant_
         // ---------------------------------------------- 1b. route (all warps)
         int re = -1;
         float rw = 0.0f;
-        if (!a.idx_in) {
+        if (!idx_in) {
             const float *row = kRouter ? lsm : a.logits + (size_t)l * E;
             auto logit_of = [&](int e) { return kRouter ? row[e] : __ldg(row + e); };
             if (kSmallK)
@@ -460,7 +455,7 @@ __global__ void __launch_bounds__(kThr, 1) decode1_kernel(const __grid_constant_
             stamp_dep<kFull>(a, l, 29, lane == 0, 0.f);
             int e = re;
             float w = rw;
-            if (a.idx_in && lane < k) { e = a.idx_in[lane]; w = a.wts_in[lane]; }
+            if (idx_in && lane < k) { e = idx_in[lane]; w = a.wts_in[lane]; }
             stamp_dep<kFull>(a, l, 2, lane == 0, w);
             bool bad = lane < k && (unsigned)e >= (unsigned)E;
             const uint8_t *base = nullptr;
@@ -631,7 +626,7 @@ __global__ void __launch_bounds__(kThr, 1) decode1_kernel(const __grid_constant_
                 // lane's float4 i) until each carries this layer's tag; every
                 // load of a round is in flight before the tags are checked (the
                 // test hook of a one-layer launch expects a tag nobody writes)
-                const uint32_t tag = xch_tag(epoch, l) ^ (a.extra_arrivals && a.L == 1 ? 1u : 0u);
+                const uint32_t tag = xch_tag(epoch, l) ^ (kFull && a.extra_arrivals && a.L == 1 ? 1u : 0u);
                 float4 q4[kHLoads];
                 unsigned pend = 0;
 #pragma unroll
@@ -844,7 +839,7 @@ hfq_status decode1_launch(const hfq4_layer *layers, int L, const float *logits, 
     a.xbuf = reinterpret_cast<uint64_t *>(xbuf); a.h = reinterpret_cast<uint64_t *>(h); a.y = y; a.y_bf16 = y_bf16; a.idx_all = idx_all; a.wts_all = wts_all;
     a.ctl = ctl; a.timeout_ns = timeout_ns; a.extra_arrivals = extra_arrivals;
     a.timeline = static_cast<unsigned long long *>(option_timeline());
-    a.L = L; a.E = E; a.k = k; a.H = H; a.I = I; a.x0_f32 = x0_f32 ? 1 : 0;
+    a.L = L; a.E = E; a.k = k; a.H = H; a.I = I;
 
     // shared-memory layout
     const int nbH = (H + kBlock - 1) / kBlock, nbI = (I + kBlock - 1) / kBlock;
@@ -876,7 +871,7 @@ hfq_status decode1_launch(const hfq4_layer *layers, int L, const float *logits, 
     const size_t smem = (size_t)a.sh_off + sizeof(D1Shared);
 
     // the instantiation for this launch, and its shared-memory limit (set once)
-    bool full = a.timeline != nullptr;
+    bool full = a.timeline != nullptr || idx_in != nullptr || extra_arrivals != 0;
     for (int l = 0; l < L; ++l) full = full || layers[l].expert_loc != nullptr;
     const int variant = (router ? 4 : 0) + (k <= kW ? 2 : 0) + (full ? 1 : 0);
     const void *const kernels[8] = {
