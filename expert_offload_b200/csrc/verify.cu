@@ -117,9 +117,10 @@ __device__ __forceinline__ Span span_of(size_t off, size_t len)
 }
 
 // Debug timeline: stamp s of layer l for this CTA (ns of %globaltimer).
+template <bool kOn>
 __device__ __forceinline__ void vstamp(const VArgs &a, int l, int s, bool who)
 {
-    if (a.timeline && who && l < a.L)
+    if (kOn && a.timeline && who && l < a.L)
         a.timeline[((size_t)blockIdx.x * a.L + l) * 32 + s] = globaltimer_ns();
 }
 
@@ -254,6 +255,10 @@ __device__ void build_pairs(VShared &sh, const VArgs &a, int l, const uint8_t *t
     __syncwarp();
 }
 
+// kFull: host-mapped experts, given routing, the debug timeline or the test
+// hook are possible; the other instantiation leaves those paths out (smaller
+// code: fewer instruction-cache misses).
+template <bool kFull>
 __global__ void __launch_bounds__(kThr, 1) verify_kernel(const __grid_constant__ VArgs a)
 {
     extern __shared__ __align__(1024) uint8_t smem[];
@@ -295,10 +300,10 @@ __global__ void __launch_bounds__(kThr, 1) verify_kernel(const __grid_constant__
 
     int stage_base = 0;                 // ring items of earlier layers (same in every warp)
     for (int l = 0; l < a.L; ++l) {
-        vstamp(a, l, 0, tid == 0);
+        vstamp<kFull>(a, l, 0, tid == 0);
         // ---------------------------------------------- 1. route, pairs, inputs
         if (warp < T) {
-            if (a.idx_in) {
+            if (kFull && a.idx_in) {
                 for (int j = lane; j < k; j += 32) {
                     int e = a.idx_in[warp * k + j];
                     if ((unsigned)e >= (unsigned)a.E) {
@@ -360,10 +365,10 @@ __global__ void __launch_bounds__(kThr, 1) verify_kernel(const __grid_constant__
                 for (int i = tid; i < kCW * T * kMaxDRows; i += kCW * 32) ysh[i] = 0.0f;
         }
         __syncthreads();
-        vstamp(a, l, 1, tid == 0);
+        vstamp<kFull>(a, l, 1, tid == 0);
         if (warp == 0) build_pairs(sh, a, l, tab);
         if (__syncthreads_or(sh.abort)) break;
-        vstamp(a, l, 2, tid == 0);
+        vstamp<kFull>(a, l, 2, tid == 0);
         const int U = sh.U, P = sh.P;
         if (a.idx_all && c == 0 && warp < T && lane < k) {
             a.idx_all[((size_t)l * T + warp) * k + lane] = sh.sel[warp][lane];
@@ -400,7 +405,7 @@ __global__ void __launch_bounds__(kThr, 1) verify_kernel(const __grid_constant__
                     const int np = min(kCW, sh.pair0[u + 1] - sh.pair0[u]);
                     if (np < kCW) mbar_arrive_cnt(&sh.empty[s], (uint32_t)(kCW - np));
                 }
-                if (!sh.uloc[u]) {
+                if (!(kFull && sh.uloc[u])) {
                     if (lane == 0) {
                         // expert bytes are read once per step: evict them first from L2
                         const uint64_t pol = l2_evict_first_policy();
@@ -432,10 +437,10 @@ __global__ void __launch_bounds__(kThr, 1) verify_kernel(const __grid_constant__
                     __syncwarp();
                     if (lane == 0) mbar_arrive(&sh.full[s]);
                 }
-                vstamp(a, l, 8, lane == 0 && i == U - 1);
-                vstamp(a, l, 10 + i, lane == 0 && i < 10);
+                vstamp<kFull>(a, l, 8, lane == 0 && i == U - 1);
+                vstamp<kFull>(a, l, 10 + i, lane == 0 && i < 10);
             }
-            vstamp(a, l, 9, lane == 0 && warp == kCW);
+            vstamp<kFull>(a, l, 9, lane == 0 && warp == kCW);
         } else {
             // ------------------------------------------ 3. gate/up items
             const int pb = lane >> 2, pq = lane & 3;
@@ -458,7 +463,7 @@ __global__ void __launch_bounds__(kThr, 1) verify_kernel(const __grid_constant__
                         note_wait(a, w, 2, l, seq);
                     }
                     ok = __shfl_sync(0xffffffffu, w, 0) != 0;
-                    vstamp(a, l, 3, lane == 0 && u == 0 && warp == 0);
+                    vstamp<kFull>(a, l, 3, lane == 0 && u == 0 && warp == 0);
                 }
                 for (; p < sh.pair0[u + 1] && ok; p += kCW) {
                     uint32_t X[32];
@@ -475,7 +480,7 @@ __global__ void __launch_bounds__(kThr, 1) verify_kernel(const __grid_constant__
                         xe = (int)es.x;
                         sxp = __uint_as_float(es.y);
                     }
-                    vstamp(a, l, 24, lane == 0 && warp == 0 && p == 0);
+                    vstamp<kFull>(a, l, 24, lane == 0 && warp == 0 && p == 0);
                     float *hrow = a.h + (size_t)sh.prow[p] * Ip + gu_lo;
                     const uint8_t *g0 = st + sg.delta, *u0 = st + up_off + su.delta;
                     for (int r0 = 0; r0 < n_gu; r0 += kGuRows) {
@@ -516,7 +521,7 @@ __global__ void __launch_bounds__(kThr, 1) verify_kernel(const __grid_constant__
                         const int i = lane >> 2;
                         if (lane < 16 && (lane & 3) == 0 && r0 + i < n_gu) hrow[r0 + i] = silu(g) * uu;
                     }
-                    vstamp(a, l, 25, lane == 0 && warp == 0 && p == 0);
+                    vstamp<kFull>(a, l, 25, lane == 0 && warp == 0 && p == 0);
                 }
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&sh.empty[s]);        // this warp is done with the stage
@@ -524,7 +529,7 @@ __global__ void __launch_bounds__(kThr, 1) verify_kernel(const __grid_constant__
             // ------------------------------------------ 4. h exchange
             unsigned *hcnt = a.ctl + kCtlH + (size_t)l * kCtlHStride;
             consumer_sync();
-            vstamp(a, l, 4, tid == 0);
+            vstamp<kFull>(a, l, 4, tid == 0);
             if (tid == 0) {
                 if (!ok) sh.abort = 1;
                 __threadfence();
@@ -535,7 +540,7 @@ __global__ void __launch_bounds__(kThr, 1) verify_kernel(const __grid_constant__
                 }
             }
             consumer_sync();
-            vstamp(a, l, 5, tid == 0);
+            vstamp<kFull>(a, l, 5, tid == 0);
             ok = ok && !sh.abort;
 
             // ------------------------------------------ 5. down items
@@ -598,7 +603,7 @@ __global__ void __launch_bounds__(kThr, 1) verify_kernel(const __grid_constant__
                         waited = true;
                         if (!ok) break;
                     }
-                    vstamp(a, l, 26, lane == 0 && warp == 0 && p == 0);
+                    vstamp<kFull>(a, l, 26, lane == 0 && warp == 0 && p == 0);
                     const uint8_t *d0 = st + sd.delta + (pc >> 2) * kBlockBytes;   // this lane's block of each row
                     const float wp = sh.pw[p];
                     float *yt = ysh + ((size_t)warp * T + sh.pt[p]) * kMaxDRows;
@@ -626,7 +631,7 @@ __global__ void __launch_bounds__(kThr, 1) verify_kernel(const __grid_constant__
                             if (pc == 0 && ri < n_d) yt[ri] += wp * v[q];
                         }
                     }
-                    vstamp(a, l, 27, lane == 0 && warp == 0 && p == 0);
+                    vstamp<kFull>(a, l, 27, lane == 0 && warp == 0 && p == 0);
                 }
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&sh.empty[s]);
@@ -638,7 +643,7 @@ __global__ void __launch_bounds__(kThr, 1) verify_kernel(const __grid_constant__
         }
         stage_base += 2 * U;
         __syncthreads();
-        vstamp(a, l, 6, tid == 0);
+        vstamp<kFull>(a, l, 6, tid == 0);
 
         // ---------------------------------------------- 6. combine, residual
         if (!sh.abort && tid < T * n_d) {
@@ -653,14 +658,14 @@ __global__ void __launch_bounds__(kThr, 1) verify_kernel(const __grid_constant__
             uint16_t *xo = last ? a.x_out : (a.xbuf ? a.xbuf + (size_t)((l + 1) & 1) * T * H : nullptr);
             if (xo) xo[o] = float_to_bf16_bits(xres[t * kMaxDRows + ri] + y);
         }
-        vstamp(a, l, 7, tid == 0);
+        vstamp<kFull>(a, l, 7, tid == 0);
         if (l + 1 < a.L) {
             __syncthreads();
             if (tid == 0) {
                 unsigned *bar = a.ctl + kCtlBar + l;
                 __threadfence();
                 red_release_gpu_add(bar, 1u);
-                if (!sh.abort && !wait_counter_ge(wc, bar, (unsigned)(G + a.extra_arrivals))) {
+                if (!sh.abort && !wait_counter_ge(wc, bar, (unsigned)(G + (kFull ? a.extra_arrivals : 0)))) {
                     sh.abort = 1;
                     note_wait(a, false, 5, l, 0);
                 }
@@ -755,17 +760,22 @@ hfq_status verify_launch(const hfq4_layer *layers, int L, const float *logits, c
     const size_t tab_b = up128((size_t)E * 9);
     fixed = xp_b + xres_b + ysh_b + hst_b + tab_b + up128(sizeof(VShared));
 
-    static int dyn_limit = 0;
+    // the instantiation for this launch and its shared-memory limit (set once)
+    bool full = a.timeline != nullptr || idx_in != nullptr || extra_arrivals != 0;
+    for (int l = 0; l < L; ++l) full = full || layers[l].expert_loc != nullptr;
+    const void *kernel = full ? (const void *)verify_kernel<true> : (const void *)verify_kernel<false>;
+    static int dyn_limits[2] = {0, 0};
+    int &dyn_limit = dyn_limits[full ? 1 : 0];
     if (!dyn_limit) {
         int dev = 0, optin = 0;
         cudaGetDevice(&dev);
         cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
         cudaFuncAttributes fa;
-        cudaError_t e = cudaFuncGetAttributes(&fa, verify_kernel);
+        cudaError_t e = cudaFuncGetAttributes(&fa, kernel);
         if (e != cudaSuccess) return fail(HFQ_ERR_CUDA, "verify kernel attributes: %s", cudaGetErrorString(e));
         int lim = optin - (int)fa.sharedSizeBytes;
         if (lim > kSmemOptin) lim = kSmemOptin;
-        e = cudaFuncSetAttribute(verify_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, lim);
+        e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, lim);
         if (e != cudaSuccess) return fail(HFQ_ERR_CUDA, "verify kernel attribute %d: %s", lim, cudaGetErrorString(e));
         dyn_limit = lim;
     }
@@ -788,7 +798,7 @@ hfq_status verify_launch(const hfq4_layer *layers, int L, const float *logits, c
     const size_t smem = (size_t)a.sh_off + sizeof(VShared);
     if (smem > (size_t)dyn_limit) return HFQ_ERR_UNSUPPORTED;
     int resident = 0;
-    cudaError_t oe = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&resident, verify_kernel, kThr, smem);
+    cudaError_t oe = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&resident, kernel, kThr, smem);
     if (oe != cudaSuccess || resident < 1) return HFQ_ERR_UNSUPPORTED;
 
     cudaLaunchConfig_t cfg = {};
@@ -802,7 +812,7 @@ hfq_status verify_launch(const hfq4_layer *layers, int L, const float *logits, c
     cfg.attrs = attrs;
     cfg.numAttrs = 1;
     void *params[] = {&a};
-    cudaError_t e = cudaLaunchKernelExC(&cfg, (const void *)verify_kernel, params);
+    cudaError_t e = cudaLaunchKernelExC(&cfg, kernel, params);
     if (e != cudaSuccess) return fail(HFQ_ERR_CUDA, "verify kernel launch: %s", cudaGetErrorString(e));
     return HFQ_OK;
 }
