@@ -509,9 +509,9 @@ def run_headline(args, rank, world, local_rank, dist):
 
 # DRAM traffic of one decode1_kernel launch on the headline workload, or None
 # while no capture of the current kernel exists (see profiles/).
-TRAFFIC_DECODE_L40 = 4 * (133848064 + 3205632)
+TRAFFIC_DECODE_L40 = 4 * (133837056 + 2886144)
 TRAFFIC_SOURCE = ("ncu dram__bytes_read.sum + dram__bytes_write.sum of one decode1_kernel<0, 1, 0> launch "
-                  "over the first 10 layers (133,848,064 + 3,205,632 B), x 4")
+                  "over the first 10 layers (133,837,056 + 2,886,144 B), x 4")
 
 
 # --------------------------------------------------------- the other configs
