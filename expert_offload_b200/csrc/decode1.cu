@@ -813,6 +813,7 @@ hfq_status decode1_launch(const hfq4_layer *layers, int L, const float *logits, 
 {
     const int H = layers[0].hidden, I = layers[0].inter, E = layers[0].n_experts;
     const int G = sm_count();
+    if (G <= 0) return fail(HFQ_ERR_CUDA, "no CUDA device");
     if (L < 1 || L > HFQ_MAX_STACK_LAYERS || k < 1 || k > kMaxK) return HFQ_ERR_UNSUPPORTED;
     if (expert_bytes(H, I) % 16) return HFQ_ERR_UNSUPPORTED;      // 16-byte aligned experts
     if (x0_f32) return HFQ_ERR_UNSUPPORTED;     // the bf16 operands need bf16-valued activations

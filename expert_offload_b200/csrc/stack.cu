@@ -820,15 +820,20 @@ size_t smem_for(int T, int H, int I, int n_stages, int maxt)
 
 }  // namespace
 
+// SMs of the current device; 0 when there is none (callers then fail with
+// HFQ_ERR_CUDA instead of sizing a grid from it).
 int sm_count()
 {
     static int n = 0;
-    if (!n) {
-        int dev = 0;
-        cudaGetDevice(&dev);
-        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    if (n <= 0) {
+        int dev = 0, v = 0;
+        if (cudaGetDevice(&dev) == cudaSuccess &&
+            cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess)
+            n = v;
+        else
+            cudaGetLastError();                 // the failed query's error is not left for a later check
     }
-    return n;
+    return n > 0 ? n : 0;
 }
 
 // Whether the persistent kernel handles this shape (else the per-layer path).

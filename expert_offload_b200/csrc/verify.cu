@@ -724,6 +724,7 @@ hfq_status verify_launch(const hfq4_layer *layers, int L, const float *logits, c
 {
     const int H = layers[0].hidden, I = layers[0].inter, E = layers[0].n_experts;
     const int G = sm_count();
+    if (G <= 0) return fail(HFQ_ERR_CUDA, "no CUDA device");
     if (L < 1 || L > HFQ_MAX_STACK_LAYERS || T < 2 || T > kMaxT || k < 1 || T * k > kMaxP)
         return HFQ_ERR_UNSUPPORTED;
     if (x0_f32 || expert_bytes(H, I) % 16) return HFQ_ERR_UNSUPPORTED;

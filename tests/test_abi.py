@@ -169,3 +169,28 @@ def test_host_arena_refuses_an_impossible_size():
             eo.hfq_host_arena_create(huge, flags)
         assert e.value.status == -7
         assert str(huge) in e.value.message
+
+
+def test_router_argument_errors_are_caught_before_launch():
+    """moe_router_logits and the routed decode stack refuse bad arguments on
+    the host (no kernel is launched on these paths)."""
+    lib = eo.lib()
+    bf16, f32 = eo.HFQ_BF16, eo.HFQ_F32
+    assert lib.moe_router_logits(None, bf16, 1, 256, 1024, bf16, 16, 1024, None) == -1
+    assert lib.moe_router_logits(1024, 7, 1, 256, 1024, bf16, 16, 1024, None) == -1          # dtype
+    assert lib.moe_router_logits(1024, bf16, 1, 252, 1024, bf16, 16, 1024, None) == -3       # hidden % 8
+    assert lib.moe_router_logits(1024, bf16, 1, 256, 1024, bf16, 513, 1024, None) == -3      # experts
+    assert lib.moe_router_logits(1026, bf16, 1, 256, 1024, bf16, 16, 1024, None) == -2       # alignment
+    lay = eo.Layer(1024, 256, 2048, 512)
+    arr = eo.layer_array([lay])
+    f = lib.hfq4_moe_decode_stack_routed
+    need = eo.hfq4_stack_workspace_bytes(1, 8, 2048, 512, 256)
+    assert f(arr, 0, 1024, bf16, 8, 1024, 1, 2048, None, None, None, None, 1024, need, None) == -1
+    assert f(arr, 1, None, bf16, 8, 1024, 1, 2048, None, None, None, None, 1024, need, None) == -1
+    assert f(arr, 1, 1024, 9, 8, 1024, 1, 2048, None, None, None, None, 1024, need, None) == -1
+    assert f(arr, 1, 1024, f32, 8, 1024, 9, 2048, None, None, None, None, 1024, need, None) == -3   # T
+    assert f(arr, 1, 1024, bf16, 8, 1026, 1, 2048, None, None, None, None, 1024, need, None) == -2  # x0
+    assert f(arr, 1, 1024, bf16, 8, 1024, 1, 2048, None, 4096, None, None, 1024, need, None) == -1  # idx without wts
+    assert f(arr, 1, 1024, bf16, 8, 1024, 1, 2048, None, None, None, None, 1024, 64, None) == -8    # workspace
+    # the routed stack needs room for the logit exchange and its own residual pair
+    assert need > eo.hfq4_moe_workspace_bytes(1, 8, 2048, 512, 256)
