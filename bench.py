@@ -59,7 +59,7 @@ def parse():
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=["decode", "verify", "offload", "prefill"], default=None,
+    ap.add_argument("--workload", choices=["decode", "verify", "offload", "prefill", "routed"], default=None,
                     help="one workload alone (default: the headline decode stack plus all others)")
     ap.add_argument("--no-suite", action="store_true", help="the headline workload only")
     ap.add_argument("--tokens", type=int, default=8, help="tokens per step (verify, prefill)")
@@ -1114,6 +1114,15 @@ def main():
         return
     import torch
     torch.cuda.set_device(local_rank)
+    if args.workload == "routed":
+        if rank == 0:
+            r = run_routed(args, args.steps, args.warmup)["decode_routed"]
+            out = {"metric": METRIC, "n_gpus": 1, "warmup": args.warmup, "higher_is_better": True,
+                   "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic"}
+            out.update(r)
+            out["config"] = {"workload": out.pop("workload")}
+            print(json.dumps(out), flush=True)
+        return
     if args.workload == "prefill":
         if rank == 0:
             r = run_prefill(args, [args.tokens], args.steps, args.warmup)
