@@ -6,10 +6,12 @@
 // token, a CTA's share of a layer is a fixed pattern: for each routed slot j,
 // rows [c*I/G, (c+1)*I/G) of the expert's gate and up matrices and rows
 // [c*H/G, (c+1)*H/G) of its down matrix (c = this CTA, G = CTAs).  Per layer:
-//   1. the eight warps route the token (each the top k of an eighth of the
-//      experts, warp 0 merging; softmax top-k, renormalised; hipfire offload
-//      explainer, opening section), reading layer l's logits only after layer
-//      l-1 has finished everywhere, and warp 0 at once issues the 2k gate/up
+//   1. the CTA routes the token (softmax top-k, renormalised; hipfire
+//      offload explainer, opening section): the warp maxima bound the k-th
+//      logit, the experts at or above the bound are ranked by unique keys
+//      (topk.cuh).  Layer l's logits are read only after layer l-1 has
+//      finished everywhere, or, with the router in the loop, computed from
+//      x_l (each CTA a share, exchanged as tagged words).  Warp 0 then issues the 2k gate/up
 //      bulk copies (1-D TMA, no multicast), lane j for slot j, into k fixed
 //      shared-memory slots with one mbarrier for gate/up and one for down per
 //      slot; warp j issues slot j's down copy once its gate/up bytes are in.  Experts
