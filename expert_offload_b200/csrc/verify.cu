@@ -10,8 +10,9 @@
 //   1. warp t routes token t (softmax top-k, renormalised; hipfire offload
 //      explainer, opening section) once layer l-1 has finished everywhere;
 //      warp 0 lists the unique experts (ascending) and their (expert, token)
-//      pairs; all threads turn the T inputs into per-64-value pieces of
-//      scaled bf16 pairs (gemv.cuh);
+//      pairs, reading the layer's expert table from shared memory (copied in
+//      while the previous layer's down items ran); all threads turn the T
+//      inputs into per-64-value pieces of scaled bf16 pairs (gemv.cuh);
 //   2. the producer warps stream one item per ring stage with 1-D bulk copies
 //      (TMA, no multicast): the gate/up share of every unique expert, then its
 //      down share; host-mapped experts are read with 16-byte loads (hipfire
